@@ -1,0 +1,200 @@
+/*
+ * CPU oracle for exact scaled-dot-product attention (float64).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * What it computes is the plain definition, written out step by step and
+ * materialising the score matrix S and the probability matrix P:
+ *
+ *   S = scale * Q K^T                ("Attention Mechanism: Computation & Memory
+ *                                     Patterns", section 1, steps 1-2;
+ *                                     "Why Attention Is Difficult to Optimize",
+ *                                     "The Attention Computation Flow")
+ *   mask: key j is visible to query i iff j <= i (causal) -- "each token can
+ *         attend only to itself and earlier tokens"; masked scores are -inf,
+ *         so their probabilities are exactly zero (same section).
+ *   P = row softmax of the masked S: p_ij = exp(s_ij) / sum over the unmasked
+ *       j' of exp(s_ij') ("From a Score Tile to Probabilities"); evaluated as
+ *       exp(s_ij - m_i) / sum exp(s_ij' - m_i) with m_i the row maximum, which
+ *       is the same number in exact arithmetic and does not overflow.
+ *   O = P V                          (section 1, step 3)
+ *   lse_i = m_i + log(sum_j exp(s_ij - m_i)) = log sum_j exp(s_ij), the row
+ *       log-sum-exp (natural log) of the scaled, masked scores.
+ *
+ * Inputs are bf16 bit patterns (uint16) widened exactly to double; scale is a
+ * double.  No blocking, fusion or reordering beyond the definition: each row
+ * block's S and P are fully materialised before O is formed.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_ROW_BLOCK 64
+
+static double bf16_to_f64(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Row softmax of n scores.  masked[j] != 0 excludes score j (probability 0).
+ * Writes p[0..n) and returns the natural-log log-sum-exp of the unmasked
+ * scores; a row with nothing unmasked gets p = 0 and returns -inf. */
+double oracle_softmax_row(const double *s, const unsigned char *masked, int n, double *p)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (!(masked && masked[j]) && s[j] > m)
+            m = s[j];
+    if (m == -INFINITY) {
+        for (int j = 0; j < n; ++j)
+            p[j] = 0.0;
+        return -INFINITY;
+    }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double e = (masked && masked[j]) ? 0.0 : exp(s[j] - m);
+        p[j] = e;
+        l += e;
+    }
+    for (int j = 0; j < n; ++j)
+        p[j] = p[j] / l;
+    return m + log(l);
+}
+
+/* One head: scores S (T x T) and probabilities P (T x T) of query rows
+ * rows[0..nrows) (all rows when rows == NULL; then nrows must equal T).
+ * q, k point at the head's [T, D] bf16 slabs.  S_out, P_out and lse_out may
+ * be NULL.  S_out holds the scaled scores before masking. */
+void oracle_head_scores_probs(const uint16_t *q, const uint16_t *k, int T, int D, int causal,
+                              double scale, const int64_t *rows, int64_t nrows,
+                              double *S_out, double *P_out, double *lse_out)
+{
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    double *p = (double *)malloc(sizeof(double) * (size_t)T);
+    unsigned char *mk = (unsigned char *)malloc((size_t)T);
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        for (int j = 0; j < T; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += bf16_to_f64(q[(size_t)i * D + c]) * bf16_to_f64(k[(size_t)j * D + c]);
+            s[j] = scale * acc;
+            mk[j] = (unsigned char)(causal && j > i);
+        }
+        double lse = oracle_softmax_row(s, mk, T, p);
+        if (S_out) memcpy(S_out + (size_t)r * T, s, sizeof(double) * (size_t)T);
+        if (P_out) memcpy(P_out + (size_t)r * T, p, sizeof(double) * (size_t)T);
+        if (lse_out) lse_out[r] = lse;
+    }
+    free(s);
+    free(p);
+    free(mk);
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int T, D, causal;
+    double scale;
+    const int64_t *heads;
+    int64_t nheads;
+    const int64_t *rows;
+    int64_t nrows;
+    double *o, *lse;
+    int64_t nitems, items_per_head;
+    int tid, nthreads;
+} job_t;
+
+/* One work item = (head, block of up to ORACLE_ROW_BLOCK requested rows):
+ * materialise that block's S and P, then O = P V for the block. */
+static void *worker(void *arg)
+{
+    job_t *jb = (job_t *)arg;
+    const int T = jb->T, D = jb->D;
+    double *S = (double *)malloc(sizeof(double) * (size_t)ORACLE_ROW_BLOCK * T);
+    double *P = (double *)malloc(sizeof(double) * (size_t)ORACLE_ROW_BLOCK * T);
+    double *L = (double *)malloc(sizeof(double) * ORACLE_ROW_BLOCK);
+    int64_t *blk_rows = (int64_t *)malloc(sizeof(int64_t) * ORACLE_ROW_BLOCK);
+    for (int64_t it = jb->tid; it < jb->nitems; it += jb->nthreads) {
+        int64_t hi = it / jb->items_per_head;
+        int64_t rb = it % jb->items_per_head;
+        int64_t bh = jb->heads ? jb->heads[hi] : hi;
+        int64_t r0 = rb * ORACLE_ROW_BLOCK;
+        int64_t nr = jb->nrows - r0;
+        if (nr > ORACLE_ROW_BLOCK) nr = ORACLE_ROW_BLOCK;
+        for (int64_t r = 0; r < nr; ++r)
+            blk_rows[r] = jb->rows ? jb->rows[r0 + r] : r0 + r;
+        const size_t head_off = (size_t)bh * (size_t)T * (size_t)D;
+        oracle_head_scores_probs(jb->q + head_off, jb->k + head_off, T, D, jb->causal, jb->scale,
+                                 blk_rows, nr, S, P, L);
+        const uint16_t *vh = jb->v + head_off;
+        for (int64_t r = 0; r < nr; ++r) {
+            size_t orow = ((size_t)hi * (size_t)jb->nrows + (size_t)(r0 + r));
+            double *out = jb->o + orow * (size_t)D;
+            for (int c = 0; c < D; ++c)
+                out[c] = 0.0;
+            const double *prow = P + (size_t)r * T;
+            for (int j = 0; j < T; ++j) {
+                double pj = prow[j];
+                if (pj == 0.0) continue; /* adds exactly nothing */
+                const uint16_t *vr = vh + (size_t)j * D;
+                for (int c = 0; c < D; ++c)
+                    out[c] += pj * bf16_to_f64(vr[c]);
+            }
+            jb->lse[orow] = L[r];
+        }
+    }
+    free(S);
+    free(P);
+    free(L);
+    free(blk_rows);
+    return NULL;
+}
+
+/* Attention forward for a subset of heads and rows.
+ *   q, k, v : bf16 bit patterns, [B*H, T, D] contiguous (head bh at bh*T*D).
+ *   heads   : flat head indices bh in [0, B*H), or NULL for all heads (then
+ *             nheads must be B*H).
+ *   rows    : query rows in [0, T), or NULL for all rows (nrows must be T).
+ *   o       : double [nheads, nrows, D];  lse : double [nheads, nrows].
+ *   nthreads: worker threads (>= 1).
+ * Returns 0, or -1 on a bad argument. */
+int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t BH, int T,
+                    int D, int causal, double scale, const int64_t *heads, int64_t nheads,
+                    const int64_t *rows, int64_t nrows, double *o, double *lse, int nthreads)
+{
+    if (!q || !k || !v || !o || !lse || BH < 1 || T < 1 || D < 1 || nheads < 1 || nrows < 1)
+        return -1;
+    if (!heads && nheads != BH) return -1;
+    if (!rows && nrows != T) return -1;
+    for (int64_t h = 0; heads && h < nheads; ++h)
+        if (heads[h] < 0 || heads[h] >= BH) return -1;
+    for (int64_t r = 0; rows && r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= T) return -1;
+    if (nthreads < 1) nthreads = 1;
+    int64_t iph = (nrows + ORACLE_ROW_BLOCK - 1) / ORACLE_ROW_BLOCK;
+    int64_t nitems = iph * nheads;
+    if (nthreads > nitems) nthreads = (int)nitems;
+    job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        job_t j = {q, k, v, T, D, causal, scale, heads, nheads, rows, nrows, o, lse, nitems, iph, t,
+                   nthreads};
+        jobs[t] = j;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        pthread_create(&th[t], NULL, worker, &jobs[t]);
+    worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(jobs);
+    free(th);
+    return 0;
+}

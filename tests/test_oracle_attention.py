@@ -1,0 +1,165 @@
+"""Pins of the oracle's attention forward: invariants the pages fix, closed
+forms, and a 50-digit brute force on tiny inputs.
+
+Pages: "Why Attention Is Difficult to Optimize" ("The Attention Computation
+Flow": scaling, causal mask "itself and earlier tokens", rows of P summing to
+1); "Attention Mechanism: Computation & Memory Patterns" (section 1: S = QK^T,
+P = softmax(S / sqrt(d_k)), O = PV).
+"""
+import math
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attn_inputs import bf16_bits, make_qkv
+
+
+def _f64(bits):
+    return bits.astype(np.uint32).__lshift__(16).view(np.float32).astype(np.float64)
+
+
+def _bits(x: torch.Tensor):
+    return bf16_bits(x.to(torch.bfloat16))
+
+
+def _rand_head(T, D, seed, mult=1.0):
+    q, k, v = make_qkv(1, 1, T, D, seed, mult)
+    return bf16_bits(q[0, 0]), bf16_bits(k[0, 0]), bf16_bits(v[0, 0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one_and_future_is_zero(causal):
+    T, D = 37, 16
+    q, k, _ = _rand_head(T, D, 5)
+    S, P, _ = oracle.head_scores_probs(q, k, causal, 1 / math.sqrt(D))
+    assert np.all(np.abs(P.sum(axis=1) - 1.0) < 1e-12)
+    if causal:
+        iu = np.triu_indices(T, 1)
+        assert np.all(P[iu] == 0.0)  # exactly zero, not merely small
+        assert np.all(P[np.tril_indices(T)] > 0.0)
+    else:
+        assert np.all(P > 0.0)
+
+
+def test_scores_are_scaled_q_dot_k_not_transposed():
+    T, D = 6, 4
+    q, k, _ = _rand_head(T, D, 11)
+    scale = 0.37
+    S, _, _ = oracle.head_scores_probs(q, k, False, scale)
+    qf, kf = _f64(q), _f64(k)
+    mpmath.mp.dps = 50
+    for i in range(T):
+        for j in range(T):
+            ref = mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(qf[i, c]) * mpmath.mpf(kf[j, c])
+                                                  for c in range(D))
+            assert abs(S[i, j] - float(ref)) < 1e-14 * max(1.0, abs(float(ref)))
+    # Q and K are not symmetric, so a transposed product would differ
+    assert not np.allclose(S, S.T)
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 64, 65, 130])
+def test_causal_row0_is_v0(T):
+    D = 8
+    q, k, v = _rand_head(T, D, 100 + T)
+    o, lse = oracle.attn_fwd(q, k, v, True, 1 / math.sqrt(D))
+    assert np.array_equal(o[0, 0], _f64(v)[0])  # exactly: P_00 = 1
+    qk = float(np.dot(_f64(q)[0], _f64(k)[0]))
+    assert abs(lse[0, 0] - qk / math.sqrt(D)) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_keys_give_prefix_means(causal):
+    T, D = 77, 8
+    q, _, v = _rand_head(T, D, 7)
+    k = np.zeros_like(q)
+    o, lse = oracle.attn_fwd(q, k, v, causal, 0.125)
+    vf = _f64(v)
+    if causal:
+        ref = np.cumsum(vf, axis=0) / np.arange(1, T + 1)[:, None]
+        ref_lse = np.log(np.arange(1, T + 1))
+    else:
+        ref = np.broadcast_to(vf.mean(axis=0), (T, D))
+        ref_lse = np.full(T, math.log(T))
+    assert np.max(np.abs(o[0] - ref)) < 1e-12
+    assert np.max(np.abs(lse[0] - ref_lse)) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_values_pass_through(causal):
+    T, D = 50, 16
+    q, k, _ = _rand_head(T, D, 8, 4.0)
+    v = _bits(torch.full((T, D), -1.75))
+    o, _ = oracle.attn_fwd(q, k, v, causal, 1 / 4)
+    assert np.max(np.abs(o + 1.75)) < 1e-12
+
+
+def test_single_token_output_is_v():
+    q, k, v = _rand_head(1, 64, 9)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, causal, 0.125)
+        assert np.array_equal(o[0, 0], _f64(v)[0])
+
+
+def test_noncausal_permutation_invariance():
+    T, D = 40, 8
+    q, k, v = _rand_head(T, D, 10)
+    perm = np.random.default_rng(0).permutation(T)
+    o1, l1 = oracle.attn_fwd(q, k, v, False, 0.3)
+    o2, l2 = oracle.attn_fwd(q, k[perm], v[perm], False, 0.3)
+    assert np.max(np.abs(o1 - o2)) < 1e-12 and np.max(np.abs(l1 - l2)) < 1e-12
+
+
+def _brute(qf, kf, vf, causal, scale):
+    """Naive formula at 50 digits, no max subtraction: o_i = sum_j e^{s_ij} v_j / sum_j e^{s_ij}."""
+    mpmath.mp.dps = 50
+    T, D = qf.shape
+    o = np.zeros((T, D))
+    lse = np.zeros(T)
+    for i in range(T):
+        js = [j for j in range(T) if not (causal and j > i)]
+        e = {}
+        for j in js:
+            s = mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(qf[i, c]) * mpmath.mpf(kf[j, c])
+                                                for c in range(D))
+            e[j] = mpmath.exp(s)
+        den = mpmath.fsum(e.values())
+        for c in range(D):
+            o[i, c] = float(mpmath.fsum(e[j] * mpmath.mpf(vf[j, c]) for j in js) / den)
+        lse[i] = float(mpmath.log(den))
+    return o, lse
+
+
+@pytest.mark.parametrize("T,D,causal,mult", [(1, 1, True, 1.0), (3, 2, True, 1.0),
+                                             (7, 4, False, 1.0), (16, 8, True, 1.0),
+                                             (16, 8, False, 4.0), (11, 5, True, 4.0)])
+def test_brute_force_tiny(T, D, causal, mult):
+    q, k, v = _rand_head(T, D, 1000 + 31 * T + D, mult)
+    scale = 1 / math.sqrt(D)
+    o, lse = oracle.attn_fwd(q, k, v, causal, scale)
+    bo, bl = _brute(_f64(q), _f64(k), _f64(v), causal, scale)
+    assert np.max(np.abs(o[0] - bo)) < 1e-13
+    assert np.max(np.abs(lse[0] - bl)) < 1e-13 * max(1.0, float(np.max(np.abs(bl))))
+
+
+def test_subsets_match_full():
+    B, H, T, D = 2, 2, 150, 16
+    q, k, v = make_qkv(B, H, T, D, 3)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    o, l = oracle.attn_fwd(qb, kb, vb, True, 0.25)
+    heads = [3, 0]
+    rows = [149, 0, 63, 64, 65, 127, 128]
+    os_, ls = oracle.attn_fwd(qb, kb, vb, True, 0.25, heads=heads, rows=rows, nthreads=3)
+    for a, h in enumerate(heads):
+        assert np.array_equal(os_[a], o[h][rows])
+        assert np.array_equal(ls[a], l[h][rows])
+
+
+def test_bad_arguments_raise():
+    q, k, v = _rand_head(8, 4, 1)
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, True, 1.0, rows=[8])
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, True, 1.0, heads=[1])
