@@ -1,0 +1,14 @@
+"""B200-native exact attention forward.
+
+The work happens in ``libattn_b200.so`` (hand-written sm_100a CUDA behind the
+C ABI in ``include/attn.h``); this package only marshals torch tensors
+(device memory and streams) into that ABI.  There is no fallback: if the
+library is missing every call raises.
+"""
+from ._lib import (AttnError, fwd, fwd_host, fwd_unfused, last_error, library_path,
+                   load_library, selftest_pv_tile, selftest_qk_tile, selftest_timeout,
+                   set_mma_order, status_str, unfused_workspace_bytes, version)
+
+__all__ = ["AttnError", "fwd", "fwd_host", "fwd_unfused", "last_error", "library_path",
+           "load_library", "selftest_pv_tile", "selftest_qk_tile", "selftest_timeout",
+           "set_mma_order", "status_str", "unfused_workspace_bytes", "version"]

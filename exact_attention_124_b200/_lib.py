@@ -1,0 +1,196 @@
+"""ctypes binding of ``libattn_b200.so`` -- argument marshalling only.
+
+Names follow the C ABI (include/attn.h, include/attn_selftest.h).  Tensors
+must already live on the current CUDA device; their ``data_ptr()`` and the
+current torch stream are handed to the library, which does all the work.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libattn_b200.so")
+_lib = None
+
+ATTN_OK = 0
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_str(code) if _lib else code} (status {code})")
+
+
+def library_path() -> str:
+    return _SO
+
+
+def load_library():
+    """Load the in-tree CUDA library; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_SO):
+        raise ImportError(f"{_SO} is missing: build it with `python -m exact_attention_124_b200.build`"
+                          " (the attention path has no fallback)")
+    lib = ctypes.CDLL(_SO)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.attn_fwd_unfused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.attn_unfused_workspace_bytes.argtypes = [I, I, I]
+    lib.attn_unfused_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_last_error.argtypes = []
+    lib.attn_status_str.argtypes = [I]
+    lib.attn_status_str.restype = ctypes.c_char_p
+    lib.attn_fused_grid_ctas.argtypes = [I, I, I, I]
+    lib.attn_version.restype = ctypes.c_char_p
+    lib.attn_selftest_qk_tile.argtypes = [P, P, P, I, P]
+    lib.attn_selftest_pv_tile.argtypes = [P, P, P, I, P]
+    lib.attn_selftest_timeout.argtypes = [I, P]
+    lib.attn_selftest_set_mma_order.argtypes = [I]
+    lib.attn_selftest_last_wait_site.argtypes = []
+    for name in ("attn_fwd", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
+                 "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
+                 "attn_selftest_timeout", "attn_selftest_set_mma_order",
+                 "attn_selftest_last_wait_site"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_str(code: int) -> str:
+    return load_library().attn_status_str(int(code)).decode()
+
+
+def version() -> str:
+    return load_library().attn_version().decode()
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(rc: int, what: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, what)
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, T, d_h] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def _want(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+def fwd(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, stream=None):
+    """Fused forward.  Returns (o bf16 [B,H,T,d_h], lse fp32 [B,H,T])."""
+    lib = load_library()
+    B, H, T, D = _shape(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t, n)
+        if tuple(t.shape) != (B, H, T, D):
+            raise ValueError("q, k, v shapes differ")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    rc = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, T, D, int(bool(causal)), float(scale), _stream(stream))
+    _check(rc, "attn_fwd")
+    return o, lse
+
+
+def unfused_workspace_bytes(B: int, H: int, T: int) -> int:
+    return int(load_library().attn_unfused_workspace_bytes(B, H, T))
+
+
+def fwd_unfused(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None,
+                s_ws=None, p_ws=None, stream=None):
+    """Three-kernel forward with S and P in device memory.
+    Returns (o, lse, s_ws, p_ws); the workspaces hold S and P ([B,H,T,T] bf16)."""
+    lib = load_library()
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    if s_ws is None:
+        s_ws = torch.empty((B, H, T, T), dtype=torch.bfloat16, device=q.device)
+    if p_ws is None:
+        p_ws = torch.empty((B, H, T, T), dtype=torch.bfloat16, device=q.device)
+    rc = lib.attn_fwd_unfused(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), s_ws.data_ptr(), p_ws.data_ptr(), B, H, T, D,
+                              int(bool(causal)), float(scale), _stream(stream))
+    _check(rc, "attn_fwd_unfused")
+    return o, lse, s_ws, p_ws
+
+
+def fwd_host(q_host, k_host, v_host, o_host, lse_host, dq, dk, dv, do_, dlse, causal: bool,
+             scale: float | None = None, stream=None):
+    """Host-buffer forward: H2D copies, the fused kernel and D2H copies, all
+    enqueued on ``stream`` by the library.  Host tensors should be pinned."""
+    lib = load_library()
+    B, H, T, D = _shape(q_host)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib.attn_fwd_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                           o_host.data_ptr(), lse_host.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                           dv.data_ptr(), do_.data_ptr(), dlse.data_ptr(), B, H, T, D,
+                           int(bool(causal)), float(scale), _stream(stream))
+    _check(rc, "attn_fwd_host")
+
+
+def last_error() -> int:
+    """Synchronise the device and return (and clear) the device status word."""
+    return int(load_library().attn_last_error())
+
+
+def last_wait_site() -> int:
+    return int(load_library().attn_selftest_last_wait_site())
+
+
+def set_mma_order(mode: int) -> int:
+    prev = load_library().attn_selftest_set_mma_order(int(mode))
+    if prev < 0:
+        raise ValueError("mode must be 0 or 1")
+    return prev
+
+
+def selftest_qk_tile(q, k, stream=None):
+    lib = load_library()
+    D = int(q.shape[-1])
+    s = torch.empty((128, 128), dtype=torch.float32, device=q.device)
+    _check(lib.attn_selftest_qk_tile(q.data_ptr(), k.data_ptr(), s.data_ptr(), D,
+                                     _stream(stream)), "attn_selftest_qk_tile")
+    return s
+
+
+def selftest_pv_tile(p, v, stream=None):
+    lib = load_library()
+    D = int(v.shape[-1])
+    o = torch.empty((128, D), dtype=torch.float32, device=v.device)
+    _check(lib.attn_selftest_pv_tile(p.data_ptr(), v.data_ptr(), o.data_ptr(), D,
+                                     _stream(stream)), "attn_selftest_pv_tile")
+    return o
+
+
+def selftest_timeout(limit_us: int, stream=None):
+    _check(load_library().attn_selftest_timeout(int(limit_us), _stream(stream)),
+           "attn_selftest_timeout")

@@ -1,0 +1,361 @@
+// attn_lib.cu -- the C ABI (include/attn.h, include/attn_selftest.h): argument
+// checks, TMA tensor maps, launches.  The whole library is this one
+// translation unit, so the device status word has a single definition.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "attn.h"
+#include "attn_selftest.h"
+#include "fused_fwd.cuh"
+#include "selftest.cuh"
+#include "unfused.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+int g_mma_order = 0;
+unsigned int g_last_where = 0;
+
+struct DeviceState {
+    bool ready = false;
+    int sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+int get_encoder()
+{
+    if (g_encode) return ATTN_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return ATTN_OK;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+           cudaSuccess;
+}
+
+// Per-device one-time set-up: device check (compute capability 10.0),
+// SM count, shared-memory opt-in of every kernel.
+int device_ready(int *sms_out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_NO_DEVICE;
+    }
+    DeviceState &st = g_dev[dev];
+    if (!st.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return ATTN_ERR_NO_DEVICE;
+        }
+        if (major != 10 || minor != 0 || sms < 1) return ATTN_ERR_NO_DEVICE;
+        if (get_encoder() != ATTN_OK) return ATTN_ERR_LAUNCH;
+        bool ok = true;
+        ok &= set_smem(attn::attn_fwd_fused_kernel<64>, attn::FusedCfg<64>::SMEM);
+        ok &= set_smem(attn::attn_fwd_fused_kernel<128>, attn::FusedCfg<128>::SMEM);
+        ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
+        ok &= set_smem(attn::s_gemm_kernel<128>, attn::K1_SMEM);
+        ok &= set_smem(attn::pv_gemm_kernel<64>, attn::PvCfg<64>::SMEM);
+        ok &= set_smem(attn::pv_gemm_kernel<128>, attn::PvCfg<128>::SMEM);
+        ok &= set_smem(attn::selftest_qk_kernel<64>, 1024 + 2 * 128 * 64 * 2 + 64);
+        ok &= set_smem(attn::selftest_qk_kernel<128>, 1024 + 2 * 128 * 128 * 2 + 64);
+        ok &= set_smem(attn::selftest_pv_kernel<64>, 1024 + 128 * 64 * 2 + 64);
+        ok &= set_smem(attn::selftest_pv_kernel<128>, 1024 + 128 * 128 * 2 + 64);
+        if (!ok) {
+            (void)cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        st.sms = sms;
+        st.ready = true;
+    }
+    if (sms_out) *sms_out = st.sms;
+    return ATTN_OK;
+}
+
+// bf16 tensor [heads, rows, inner] as a 3-D TMA map with 128-byte swizzle and
+// a box of (64, box_rows, 1) elements; out-of-range rows read as zero.
+int make_map(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uint64_t heads,
+             uint32_t box_rows)
+{
+    cuuint64_t dims[3] = {inner, rows, heads};
+    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// Host-side checks shared by every forward entry point; no CUDA call here.
+int validate(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
+             int H, int T, int d_h, int causal, float scale)
+{
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    if (d_h != 64 && d_h != 128) return ATTN_ERR_UNSUPPORTED_DH;
+    if (B < 1 || H < 1 || T < 1) return ATTN_ERR_BAD_SHAPE;
+    const long long bh = (long long)B * H;
+    if (bh * (long long)T > (long long)INT_MAX || T > INT_MAX - 256) return ATTN_ERR_BAD_SHAPE;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse))
+        return ATTN_ERR_ALIGN;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_BAD_SCALE;
+    if (causal != 0 && causal != 1) return ATTN_ERR_BAD_ARG;
+    return ATTN_OK;
+}
+
+int launch_status()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D>
+int launch_fused(const void *q, const void *k, const void *v, void *o, float *lse, int BH, int T,
+                 int causal, float scale, cudaStream_t stream, int sms)
+{
+    using C = attn::FusedCfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, BH, 128) ||
+        make_map(&mv, v, D, T, BH, 128))
+        return ATTN_ERR_LAUNCH;
+    attn::FusedParams p;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.BH = BH;
+    p.T = T;
+    p.causal = causal;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.nqb = (T + 255) / 256;
+    p.units = BH * p.nqb;
+    p.nkv = (T + 127) / 128;
+    p.order_mode = g_mma_order;
+    p.limit_ns = kWaitLimitNs;
+    const int grid = p.units < sms ? p.units : sms;
+    attn::attn_fwd_fused_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    return launch_status();
+}
+
+template <int D>
+int launch_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
+                   void *p_ws, int BH, int T, int causal, float scale, cudaStream_t stream)
+{
+    CUtensorMap mq, mk, mp, mv;
+    if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, BH, 128) ||
+        make_map(&mp, p_ws, T, T, BH, 128) || make_map(&mv, v, D, T, BH, 64))
+        return ATTN_ERR_LAUNCH;
+    attn::UnfusedParams p;
+    p.BH = BH;
+    p.T = T;
+    p.causal = causal;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.limit_ns = kWaitLimitNs;
+    auto *S = static_cast<__nv_bfloat16 *>(s_ws);
+    auto *P = static_cast<__nv_bfloat16 *>(p_ws);
+    attn::s_gemm_kernel<D><<<dim3(T / 128, T / 128, BH), 128, attn::K1_SMEM, stream>>>(mq, mk, S,
+                                                                                      p);
+    if (launch_status()) return ATTN_ERR_LAUNCH;
+    const long long rows = (long long)BH * T;
+    attn::softmax_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(S, P, lse, p);
+    if (launch_status()) return ATTN_ERR_LAUNCH;
+    attn::pv_gemm_kernel<D><<<dim3(T / 128, BH), 128, attn::PvCfg<D>::SMEM, stream>>>(
+        mp, mv, static_cast<__nv_bfloat16 *>(o), p);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
+             int d_h, int causal, float scale, void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    int sms = 0;
+    if ((rc = device_ready(&sms))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64 ? launch_fused<64>(q, k, v, o, lse, B * H, T, causal, scale, s, sms)
+                     : launch_fused<128>(q, k, v, o, lse, B * H, T, causal, scale, s, sms);
+}
+
+size_t attn_unfused_workspace_bytes(int B, int H, int T)
+{
+    if (B < 1 || H < 1 || T < 1) return 0;
+    const unsigned long long n = (unsigned long long)B * H * T * (unsigned long long)T * 2ull;
+    return (size_t)n;
+}
+
+int attn_fwd_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
+                     void *p_ws, int B, int H, int T, int d_h, int causal, float scale,
+                     void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    if (!s_ws || !p_ws) return ATTN_ERR_NULL;
+    if (misaligned(s_ws) || misaligned(p_ws)) return ATTN_ERR_ALIGN;
+    if (T % 128 != 0 || (long long)B * H > 65535) return ATTN_ERR_BAD_SHAPE;
+    if ((rc = device_ready(nullptr))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s)
+                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s);
+}
+
+int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                  float *lse_host, void *dq, void *dk, void *dv, void *do_, float *dlse, int B,
+                  int H, int T, int d_h, int causal, float scale, void *stream)
+{
+    if (!q_host || !k_host || !v_host || !o_host || !lse_host) return ATTN_ERR_NULL;
+    int rc = validate(dq, dk, dv, do_, dlse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    if ((rc = device_ready(nullptr))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)B * H * T * d_h * 2;
+    const size_t nl = (size_t)B * H * T * sizeof(float);
+    if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    if ((rc = attn_fwd(dq, dk, dv, do_, dlse, B, H, T, d_h, causal, scale, stream))) return rc;
+    if (cudaMemcpyAsync(o_host, do_, n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse_host, dlse, nl, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+
+int attn_last_error(void)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    unsigned int v = 0, w = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, attn::g_status, sizeof v) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&w, attn::g_status_where, sizeof w) != cudaSuccess ||
+        cudaMemcpyToSymbol(attn::g_status, &zero, sizeof zero) != cudaSuccess ||
+        cudaMemcpyToSymbol(attn::g_status_where, &zero, sizeof zero) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    g_last_where = w;
+    return (int)v;
+}
+
+const char *attn_status_str(int status)
+{
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULL: return "null pointer";
+        case ATTN_ERR_UNSUPPORTED_DH: return "unsupported head dimension (64 or 128)";
+        case ATTN_ERR_BAD_SHAPE: return "bad shape";
+        case ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ATTN_ERR_BAD_SCALE: return "scale not finite and positive";
+        case ATTN_ERR_LAUNCH: return "CUDA launch or runtime error";
+        case ATTN_ERR_TIMEOUT: return "device wait timed out";
+        case ATTN_ERR_NO_DEVICE: return "no sm_100 device";
+        case ATTN_ERR_BAD_ARG: return "bad argument";
+        default: return "unknown status";
+    }
+}
+
+int attn_fused_grid_ctas(int B, int H, int T, int d_h)
+{
+    if (B < 1 || H < 1 || T < 1 || (d_h != 64 && d_h != 128)) return 0;
+    int sms = 0;
+    if (device_ready(&sms)) return 0;
+    const long long units = (long long)B * H * ((T + 255) / 256);
+    return (int)(units < sms ? units : sms);
+}
+
+const char *attn_version(void) { return "0.1.0"; }
+
+// ------------------------------------------------------------------ self-tests
+int attn_selftest_qk_tile(const void *q, const void *k, float *s, int d_h, void *stream)
+{
+    if (!q || !k || !s) return ATTN_ERR_NULL;
+    if (d_h != 64 && d_h != 128) return ATTN_ERR_UNSUPPORTED_DH;
+    if (misaligned(q) || misaligned(k) || misaligned(s)) return ATTN_ERR_ALIGN;
+    int rc = device_ready(nullptr);
+    if (rc) return rc;
+    CUtensorMap mq, mk;
+    if (make_map(&mq, q, d_h, 128, 1, 128) || make_map(&mk, k, d_h, 128, 1, 128))
+        return ATTN_ERR_LAUNCH;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d_h == 64)
+        attn::selftest_qk_kernel<64><<<1, 128, 1024 + 2 * 128 * 64 * 2 + 64, st>>>(mq, mk, s,
+                                                                                 kWaitLimitNs);
+    else
+        attn::selftest_qk_kernel<128><<<1, 128, 1024 + 2 * 128 * 128 * 2 + 64, st>>>(mq, mk, s,
+                                                                                   kWaitLimitNs);
+    return launch_status();
+}
+
+int attn_selftest_pv_tile(const void *p, const void *v, float *o, int d_h, void *stream)
+{
+    if (!p || !v || !o) return ATTN_ERR_NULL;
+    if (d_h != 64 && d_h != 128) return ATTN_ERR_UNSUPPORTED_DH;
+    if (misaligned(p) || misaligned(v) || misaligned(o)) return ATTN_ERR_ALIGN;
+    int rc = device_ready(nullptr);
+    if (rc) return rc;
+    CUtensorMap mv;
+    if (make_map(&mv, v, d_h, 128, 1, 128)) return ATTN_ERR_LAUNCH;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const auto *pp = static_cast<const __nv_bfloat16 *>(p);
+    if (d_h == 64)
+        attn::selftest_pv_kernel<64><<<1, 128, 1024 + 128 * 64 * 2 + 64, st>>>(pp, mv, o,
+                                                                             kWaitLimitNs);
+    else
+        attn::selftest_pv_kernel<128><<<1, 128, 1024 + 128 * 128 * 2 + 64, st>>>(pp, mv, o,
+                                                                               kWaitLimitNs);
+    return launch_status();
+}
+
+int attn_selftest_timeout(int limit_us, void *stream)
+{
+    if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_BAD_ARG;
+    int rc = device_ready(nullptr);
+    if (rc) return rc;
+    attn::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_us * 1000ull);
+    return launch_status();
+}
+
+int attn_selftest_set_mma_order(int mode)
+{
+    if (mode != 0 && mode != 1) return -1;
+    const int prev = g_mma_order;
+    g_mma_order = mode;
+    return prev;
+}
+
+int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
+
+}  // extern "C"

@@ -1,0 +1,501 @@
+// fused_fwd.cuh -- fused exact attention forward for B200 (sm_100a).
+//
+// What it computes (per head, Q/K/V of T x d_h): O = softmax(mask(scale*QK^T)) V
+// and the row log-sum-exp, as defined in "Why Attention Is Difficult to
+// Optimize" ("The Attention Computation Flow") and "Attention Mechanism:
+// Computation & Memory Patterns" (section 1).  How: the IO-aware form of that
+// page's section 3 -- Q/K/V tiles staged on chip, each score tile scaled and
+// causally masked in place from query/key indices ("From a Score Tile to
+// Probabilities"), and an online softmax that carries a running maximum, a
+// running normaliser and a consistently rescaled P.V accumulator ("FlashAttention
+// -- avoid writing the giant intermediate", "Tiling and an incremental
+// normalization").  The T x T matrices S and P never leave the SM: S lives in
+// tensor memory (TMEM), P is written back over it as bf16 and read from there
+// by the second MMA.
+//
+// B200 mapping (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax warpgroup for query tile 1 (the two tiles ping-pong, so one
+//              tile's exponentials overlap the other tile's MMAs)
+//   warp 8     MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T (smem x smem)
+//              and O_t += P_t V_j (tmem x smem); allocates/frees TMEM
+//   warp 9     TMA producer (one thread): Q tiles, then K_j / V_j into an
+//              NSTAGE-deep shared-memory ring, in the order the MMA consumes them
+// A work unit is (head, 256 query rows); units are handed out longest-first
+// (causal cost grows with the query block) in a serpentine order over CTAs.
+//
+// TMEM (512 columns x 128 lanes x 32 bit):
+//   S_0 / P_0 : columns [0, 128)     S_1 / P_1 : [128, 256)
+//   O_0       : [256, 256 + d_h)     O_1       : [256 + d_h, 256 + 2 d_h)
+// Online softmax in the log2 domain: s2 = s * scale * log2(e); the running
+// maximum m only moves when a row's new maximum exceeds it by more than
+// RESCALE_TAU (2^8 headroom keeps p <= 256), so the O rescale (a TMEM
+// read-modify-write) is rare; the final O = acc / l and lse = (m + log2 l) ln 2
+// are exact for any m, stale or not.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+constexpr float RESCALE_TAU = 8.0f;
+
+struct FusedParams {
+    __nv_bfloat16 *o;
+    float *lse;
+    int BH;
+    int T;
+    int causal;
+    float c_log2;  // scale * log2(e)
+    int nqb;       // query blocks of 256 rows per head
+    int units;     // BH * nqb
+    int nkv;       // key/value tiles of 128 per head
+    int order_mode;
+    unsigned long long limit_ns;
+};
+
+template <int D>
+struct FusedCfg {
+    static_assert(D == 64 || D == 128, "d_h must be 64 or 128");
+    static constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
+    static constexpr int BN = 128;                 // keys per K/V tile
+    static constexpr int KB = D / 64;              // 128-byte column blocks per row
+    static constexpr int SUB = 128 * 128;          // one 128-row x 128-byte block
+    static constexpr int TILE = BN * D * 2;        // bytes of one Q, K or V tile
+    static constexpr int NSTAGE = (D == 64) ? 8 : 4;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = 2 * TILE;
+    static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
+    static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+    static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TM_S = 0;            // + 128 * t
+    static constexpr uint32_t TM_O = 256;          // + D * t
+    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+};
+
+// Wait codes recorded with a timeout (which barrier gave up).
+enum : unsigned int {
+    W_QFULL = 1, W_QEMPTY, W_KVFULL, W_KVEMPTY, W_SFULL, W_PFULL, W_PVDONE, W_DRAIN
+};
+
+struct UnitInfo {
+    int bh, i0;
+    int n[2];
+    int niter;
+};
+
+// k-th unit of this CTA in the serpentine, longest-first order; false when
+// the CTA has no k-th unit (callers stop at the first k with k*G >= units and
+// skip the holes of the last round).
+__device__ __forceinline__ bool unit_of(const FusedParams &p, int k, UnitInfo &u)
+{
+    const long long G = gridDim.x;
+    const long long c = blockIdx.x;
+    const long long idx = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+    if (idx >= p.units) return false;
+    const int level = (int)(idx / p.BH);
+    u.bh = (int)(idx % p.BH);
+    const int qb = p.causal ? (p.nqb - 1 - level) : level;
+    u.i0 = qb * 256;
+    for (int t = 0; t < 2; ++t) {
+        const int r0 = u.i0 + 128 * t;
+        if (r0 >= p.T) {
+            u.n[t] = 0;
+        } else if (p.causal) {
+            const int last = r0 / 128 + 1;
+            u.n[t] = last < p.nkv ? last : p.nkv;
+        } else {
+            u.n[t] = p.nkv;
+        }
+    }
+    u.niter = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
+    return true;
+}
+
+__device__ __forceinline__ bool more_units(const FusedParams &p, int k)
+{
+    return (long long)k * gridDim.x < p.units;
+}
+
+struct Ring {
+    uint32_t idx = 0, phase = 0;
+    template <int N>
+    __device__ __forceinline__ void advance()
+    {
+        if (++idx == (uint32_t)N) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const FusedParams p)
+{
+    using C = FusedCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the 128-byte-swizzled tiles
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+
+    const uint32_t sQ = base + C::OFF_Q;
+    const uint32_t sKV = base + C::OFF_KV;
+    const uint32_t bar0 = base + C::OFF_BAR;
+    const uint32_t b_qfull = bar0;                          // [2]
+    const uint32_t b_qempty = bar0 + 16;                    // [2]
+    const uint32_t b_kvfull = bar0 + 32;                    // [NSTAGE]
+    const uint32_t b_kvempty = b_kvfull + 8 * C::NSTAGE;    // [NSTAGE]
+    const uint32_t b_sfull = b_kvempty + 8 * C::NSTAGE;     // [2]
+    const uint32_t b_pfull = b_sfull + 16;                  // [2]
+    const uint32_t b_pvdone = b_pfull + 16;                 // [2]
+    const uint32_t b_drain = b_pvdone + 16;                 // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_qfull, 1);
+        mbar_init(b_qfull + 8, 1);
+        mbar_init(b_qempty, 1);
+        mbar_init(b_qempty + 8, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(b_kvfull + 8 * s, 1);
+            mbar_init(b_kvempty + 8 * s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(b_sfull + 8 * t, 1);
+            mbar_init(b_pfull + 8 * t, 128);
+            mbar_init(b_pvdone + 8 * t, 1);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 9 && lane == 0) {
+        tma_prefetch_map(&tmQ);
+        tma_prefetch_map(&tmK);
+        tma_prefetch_map(&tmV);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t lim = p.limit_ns;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol_q = policy_evict_first();
+            const uint64_t pol_kv = policy_evict_last();
+            Ring ring;
+            uint32_t qph[2] = {0u, 0u};
+            uint32_t armed = 0u, armed_par = 0u;      // bit s: slot s has a load in flight / its parity
+            uint32_t q_armed = 0u, q_armed_par = 0u;  // bit t: same for the Q tiles
+            bool ok = true;
+            auto load_kv = [&](const CUtensorMap *map, int j, int bh) -> bool {
+                const uint32_t s = ring.idx;
+                if (!mbar_wait(b_kvempty + 8 * s, ring.phase ^ 1u, lim, W_KVEMPTY, abort_flag)) return false;
+                mbar_arrive_expect_tx(b_kvfull + 8 * s, C::TILE);
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (ring.phase << s);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(sKV + s * C::TILE + kb * C::SUB, map, b_kvfull + 8 * s, 64 * kb,
+                                128 * j, bh, pol_kv);
+                ring.advance<C::NSTAGE>();
+                return true;
+            };
+            for (int k = 0; ok && more_units(p, k); ++k) {
+                UnitInfo u;
+                if (!unit_of(p, k, u)) continue;
+                if (*abort_flag) { ok = false; break; }
+                #pragma unroll
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (u.n[t] == 0) continue;
+                    if (!mbar_wait(b_qempty + 8 * t, qph[t] ^ 1u, lim, W_QEMPTY, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(b_qfull + 8 * t, C::TILE);
+                    q_armed |= 1u << t;
+                    q_armed_par = (q_armed_par & ~(1u << t)) | (qph[t] << t);
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_3d(sQ + t * C::TILE + kb * C::SUB, &tmQ, b_qfull + 8 * t, 64 * kb,
+                                    u.i0 + 128 * t, u.bh, pol_q);
+                    qph[t] ^= 1u;
+                }
+                if (!ok) break;
+                ok = load_kv(&tmK, 0, u.bh);
+                for (int j = 1; ok && j < u.niter; ++j) {
+                    ok = load_kv(&tmK, j, u.bh);
+                    if (ok) ok = load_kv(&tmV, j - 1, u.bh);
+                }
+                if (ok) ok = load_kv(&tmV, u.niter - 1, u.bh);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                // let every copy still in flight land before the CTA exits
+                for (int s = 0; s < C::NSTAGE; ++s)
+                    if ((armed >> s) & 1u)
+                        mbar_wait(b_kvfull + 8 * s, (armed_par >> s) & 1u, lim, W_KVFULL);
+                for (int t = 0; t < 2; ++t)
+                    if ((q_armed >> t) & 1u)
+                        mbar_wait(b_qfull + 8 * t, (q_armed_par >> t) & 1u, lim, W_QFULL);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            Ring ring;
+            uint32_t qph[2] = {0u, 0u};
+            uint32_t pph[2] = {0u, 0u};
+            uint32_t drain_ph = 0;
+            bool issued_any = false;
+            bool ok = true;
+            const uint32_t tS[2] = {tmem + C::TM_S, tmem + C::TM_S + 128};
+            const uint32_t tO[2] = {tmem + C::TM_O, tmem + C::TM_O + D};
+
+            auto drain = [&]() -> bool {  // wait for every MMA issued so far
+                tc_commit(b_drain);
+                const bool r = mbar_wait(b_drain, drain_ph, lim, W_DRAIN);
+                drain_ph ^= 1u;
+                return r;
+            };
+            auto qk = [&](int t, uint32_t kslot) {
+                const uint32_t qa = sQ + t * C::TILE;
+                const uint32_t kbse = sKV + kslot * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::SUB + (kk & 3) * 32;
+                    mma_ss(tS[t], sw128_desc(qa + off, 16, 1024), sw128_desc(kbse + off, 16, 1024),
+                           C::IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto pv = [&](int t, uint32_t vslot, bool acc) {
+                const uint32_t vb = sKV + vslot * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tO[t], tS[t] + 8 * kk, sw128_desc(vb + kk * 2048, C::SUB, 1024),
+                           C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            };
+
+            for (int k = 0; ok && more_units(p, k); ++k) {
+                UnitInfo u;
+                if (!unit_of(p, k, u)) continue;
+                #pragma unroll
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (u.n[t] == 0) continue;
+                    ok = mbar_wait(b_qfull + 8 * t, qph[t], lim, W_QFULL, abort_flag);
+                    qph[t] ^= 1u;
+                }
+                if (!ok) break;
+                // K_0: first score tiles
+                uint32_t ks = ring.idx;
+                if (!(ok = mbar_wait(b_kvfull + 8 * ks, ring.phase, lim, W_KVFULL, abort_flag))) break;
+                ring.advance<C::NSTAGE>();
+                tc_fence_after_sync();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (u.n[t] == 0) continue;
+                    if (p.order_mode == 1 && issued_any && !(ok = drain())) break;
+                    qk(t, ks);
+                    issued_any = true;
+                    tc_commit(b_sfull + 8 * t);
+                    if (u.n[t] == 1) tc_commit(b_qempty + 8 * t);
+                }
+                if (!ok) break;
+                tc_commit(b_kvempty + 8 * ks);
+                for (int j = 1; ok && j < u.niter; ++j) {
+                    ks = ring.idx;
+                    if (!(ok = mbar_wait(b_kvfull + 8 * ks, ring.phase, lim, W_KVFULL, abort_flag))) break;
+                    ring.advance<C::NSTAGE>();
+                    const uint32_t vs = ring.idx;
+                    if (!(ok = mbar_wait(b_kvfull + 8 * vs, ring.phase, lim, W_KVFULL, abort_flag))) break;
+                    ring.advance<C::NSTAGE>();
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (j - 1 < u.n[t]) {  // O_t += P_t(j-1) V_{j-1}
+                            if (!(ok = mbar_wait(b_pfull + 8 * t, pph[t], lim, W_PFULL, abort_flag))) break;
+                            pph[t] ^= 1u;
+                            tc_fence_after_sync();
+                            pv(t, vs, j - 1 > 0);
+                            if (j - 1 == u.n[t] - 1) tc_commit(b_pvdone + 8 * t);
+                        }
+                        if (j < u.n[t]) {      // S_t = Q_t K_j^T
+                            if (p.order_mode == 1 && !(ok = drain())) break;
+                            qk(t, ks);
+                            tc_commit(b_sfull + 8 * t);
+                            if (j == u.n[t] - 1) tc_commit(b_qempty + 8 * t);
+                        }
+                    }
+                    if (!ok) break;
+                    tc_commit(b_kvempty + 8 * ks);
+                    tc_commit(b_kvempty + 8 * vs);
+                }
+                if (!ok) break;
+                const uint32_t vs = ring.idx;
+                if (!(ok = mbar_wait(b_kvfull + 8 * vs, ring.phase, lim, W_KVFULL, abort_flag))) break;
+                ring.advance<C::NSTAGE>();
+                tc_fence_after_sync();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (u.niter - 1 < u.n[t]) {
+                        if (!(ok = mbar_wait(b_pfull + 8 * t, pph[t], lim, W_PFULL, abort_flag))) break;
+                        pph[t] ^= 1u;
+                        tc_fence_after_sync();
+                        pv(t, vs, u.niter - 1 > 0);
+                        tc_commit(b_pvdone + 8 * t);
+                    }
+                }
+                if (!ok) break;
+                tc_commit(b_kvempty + 8 * vs);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                drain();  // every issued MMA finishes before TMEM is freed
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = warp >> 2;          // query tile 0 or 1
+        const int wq = warp & 3;          // TMEM lane quarter
+        const int rit = wq * 32 + lane;   // row in tile == TMEM lane
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::TM_S + 128 * t;
+        const uint32_t tO = tmem + lane_off + C::TM_O + D * t;
+        const float cl2 = p.c_log2;
+        uint32_t sph = 0, oph = 0;
+        bool ok = true;
+        for (int k = 0; ok && more_units(p, k); ++k) {
+            UnitInfo u;
+            if (!unit_of(p, k, u)) continue;
+            const int nt = u.n[t];
+            if (nt == 0) continue;
+            const int r0 = u.i0 + 128 * t;
+            const int row = r0 + rit;
+            float m = -INFINITY;  // running max, log2 units
+            float l = 0.f;        // running normaliser
+            for (int j = 0; j < nt; ++j) {
+                bool w = mbar_wait(b_sfull + 8 * t, sph, lim, W_SFULL, abort_flag);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                sph ^= 1u;
+                tc_fence_after_sync();
+                float s[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + 32 * c, r);
+                    tmem_wait_ld_regs(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+                }
+                const int key0 = 128 * j;
+                const bool need_mask = (p.causal && key0 + 127 > r0) || (key0 + 128 > p.T);
+                if (need_mask) {
+                    const int lim_key = p.causal ? min(row, p.T - 1) : p.T - 1;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (key0 + c > lim_key) s[c] = -INFINITY;
+                }
+                float mx[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+                for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+                const float rowmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float cand = rowmax * cl2;
+                float alpha = 1.f;
+                bool resc = false;
+                if (j == 0) {
+                    m = cand;
+                } else if (cand > m + RESCALE_TAU) {
+                    alpha = fast_exp2(m - cand);
+                    m = cand;
+                    resc = true;
+                }
+                if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tO + 32 * c, r);
+                        tmem_wait_ld_regs(r);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(tO + 32 * c, r);
+                    }
+                }
+                l *= alpha;
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float p0 = fast_exp2(fmaf(s[64 * h + 2 * i], cl2, neg_m));
+                        const float p1 = fast_exp2(fmaf(s[64 * h + 2 * i + 1], cl2, neg_m));
+                        ls[(2 * i) & 3] += p0;
+                        ls[(2 * i + 1) & 3] += p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(tS + 32 * h, pk);
+                }
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(b_pfull + 8 * t);
+            }
+            if (!ok) break;
+            // epilogue: O = acc / l, lse = (m + log2 l) ln 2
+            bool w = mbar_wait(b_pvdone + 8 * t, oph, lim, W_PVDONE, abort_flag);
+            ok = __all_sync(0xffffffffu, w);
+            if (!ok) break;
+            oph ^= 1u;
+            tc_fence_after_sync();
+            const float inv_l = 1.f / l;
+            const size_t orow = (size_t)u.bh * (size_t)p.T + (size_t)row;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + 32 * c, r);
+                tmem_wait_ld_regs(r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
+                                        __uint_as_float(r[2 * i + 1]) * inv_l);
+                if (row < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + orow * D + 32 * c);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+            if (row < p.T) p.lse[orow] = (m + fast_log2(l)) * 0.69314718055994530942f;
+            tc_fence_before_sync();
+        }
+        if (!ok) *abort_flag = 1;
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 8) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace attn

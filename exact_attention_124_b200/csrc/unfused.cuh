@@ -1,0 +1,324 @@
+// unfused.cuh -- the materialised three-kernel attention forward.
+//
+// "Why Attention Is Difficult to Optimize", section "Storing and Rereading
+// Large Intermediate Matrices": the kernel computing QK^T stores the score
+// matrix S and finishes; the next kernel reads S, scales, masks and applies
+// softmax and stores P; the last kernel reads P and multiplies it by V.  S and
+// P are T x T per head at 2 bytes per value (bf16), so this path moves
+// 2 * 2 * T^2 * 2 bytes per head through device memory that the fused kernel
+// never touches.  It exists to measure that traffic.
+//
+//   K1 s_gemm_kernel     S = Q K^T   (tcgen05, 128x128 tiles, TMA operands)
+//   K2 softmax_kernel    P = softmax(mask(scale * S)), lse   (one warp per row,
+//                        warp-shuffle reduction of (max, sum) pairs)
+//   K3 pv_gemm_kernel    O = P V     (tcgen05, 128 x d_h tiles, 4-stage TMA ring)
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+struct UnfusedParams {
+    int BH, T, causal;
+    float c_log2;
+    unsigned long long limit_ns;
+};
+
+enum : unsigned int { W_K1 = 32, W_K3_FULL, W_K3_EMPTY, W_K3_DONE };
+
+// K1 asks for the d_h = 128 footprint at both head sizes: at most three CTAs
+// per SM, so their 3 x 128 TMEM columns always fit in the SM's 512.
+constexpr int K1_SMEM = 1024 + 2 * 128 * 128 * 2 + 64;
+
+// ---------------------------------------------------------------------------
+// K1: one CTA per 128 x 128 tile of S (grid: T/128 key tiles, T/128 query
+// tiles, B*H heads); 128 threads.  S written raw (unscaled) as bf16.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128)
+    s_gemm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  __nv_bfloat16 *S, const UnfusedParams p)
+{
+    constexpr int KB = D / 64, SUB = 128 * 128, TILE = 128 * D * 2;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base, sK = base + TILE;
+    const uint32_t b_load = base + 2 * TILE, b_mma = b_load + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + 2 * TILE + 16);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_load, 1);
+        mbar_init(b_mma, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(smem_addr(tmem_slot), 128);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        const uint64_t pol = policy_evict_last();
+        mbar_arrive_expect_tx(b_load, 2 * TILE);
+        for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(sQ + kb * SUB, &tmQ, b_load, 64 * kb, m0, bh, pol);
+            tma_load_3d(sK + kb * SUB, &tmK, b_load, 64 * kb, n0, bh, pol);
+        }
+        ok = mbar_wait(b_load, 0, p.limit_ns, W_K1);
+        if (ok) {
+            tc_fence_after_sync();
+            constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * SUB + (kk & 3) * 32;
+                mma_ss(tmem, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024), idesc,
+                       kk > 0 ? 1u : 0u);
+            }
+        }
+        tc_commit(b_mma);  // also covers the case with no MMA issued
+    }
+    __syncwarp();
+    const bool w = mbar_wait(b_mma, 0, p.limit_ns, W_K1);
+    ok = __all_sync(0xffffffffu, w) && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    if (ok) {
+        tc_fence_after_sync();
+        const int row = m0 + warp * 32 + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+        __nv_bfloat16 *dst_row = S + ((size_t)bh * p.T + row) * (size_t)p.T + n0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + 32 * c, r);
+            tmem_wait_ld_regs(r);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst_row + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------------------
+// K2: row softmax, one warp per query row, 8 rows per 256-thread CTA.
+// Pass 1 reads the row once (16-byte loads) and keeps a per-lane running
+// (max, sum) in the log2 domain; a butterfly of warp shuffles merges the 32
+// pairs.  Pass 2 re-reads the row (L2-resident by then) and writes
+// P = exp2(s * scale * log2e - m) / l, exactly 0 where masked.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void merge_ml(float &m, float &l, float m2, float l2)
+{
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;  // both empty
+    l = l * fast_exp2(m - mn) + l2 * fast_exp2(m2 - mn);
+    m = mn;
+}
+
+__global__ void __launch_bounds__(256)
+    softmax_kernel(const __nv_bfloat16 *__restrict__ S, __nv_bfloat16 *__restrict__ P,
+                   float *__restrict__ lse, const UnfusedParams p)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long grow = (long long)blockIdx.x * 8 + warp;  // flat row over B*H*T
+    if (grow >= (long long)p.BH * p.T) return;
+    const int row = (int)(grow % p.T);
+    const int T = p.T;
+    const float c = p.c_log2;
+    const int lim_key = p.causal ? row : T - 1;
+    const uint4 *src = reinterpret_cast<const uint4 *>(S + grow * (long long)T);
+    uint4 *dst = reinterpret_cast<uint4 *>(P + grow * (long long)T);
+    const int nchunk = T / 8;
+
+    float m = -INFINITY, l = 0.f;
+    for (int ch = lane; ch < nchunk; ch += 32) {
+        const uint4 v = src[ch];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16) * c;
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * c;
+        }
+        float cm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (ch * 8 + i > lim_key) x[i] = -INFINITY;
+            cm = fmaxf(cm, x[i]);
+        }
+        if (cm == -INFINITY) continue;
+        const float mn = fmaxf(m, cm);
+        float add = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) add += fast_exp2(x[i] - mn);
+        l = l * fast_exp2(m - mn) + add;
+        m = mn;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
+        merge_ml(m, l, m2, l2);
+    }
+    const float inv_l = 1.f / l;
+    for (int ch = lane; ch < nchunk; ch += 32) {
+        const uint4 v = src[ch];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int k0 = ch * 8 + 2 * i;
+            const float a = (k0 > lim_key)
+                                ? 0.f
+                                : fast_exp2(__uint_as_float(w[i] << 16) * c - m) * inv_l;
+            const float b = (k0 + 1 > lim_key)
+                                ? 0.f
+                                : fast_exp2(__uint_as_float(w[i] & 0xFFFF0000u) * c - m) * inv_l;
+            o[i] = pack_bf16x2(a, b);
+        }
+        dst[ch] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) lse[grow] = (m + fast_log2(l)) * 0.69314718055994530942f;
+}
+
+// ---------------------------------------------------------------------------
+// K3: O = P V, one CTA per 128 query rows of one head (grid: T/128, B*H);
+// 128 threads: thread 0 produces (TMA), thread 32 issues MMAs, all four warps
+// run the epilogue.  Keys advance 64 at a time through a 4-stage ring of
+// (P chunk 128 x 64, V chunk 64 x d_h).
+// ---------------------------------------------------------------------------
+template <int D>
+struct PvCfg {
+    static constexpr int KB = D / 64;
+    static constexpr int P_BYTES = 128 * 128;    // 128 rows x 64 keys x 2 B
+    static constexpr int V_SUB = 64 * 128;       // 64 keys x 64 d x 2 B
+    static constexpr int V_BYTES = KB * V_SUB;
+    static constexpr int STAGE = P_BYTES + V_BYTES;
+    static constexpr int NST = 4;
+    static constexpr int SMEM = 1024 + NST * STAGE + 2 * NST * 8 + 8 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    pv_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmV,
+                   __nv_bfloat16 *O, const UnfusedParams p)
+{
+    using C = PvCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t b_full = base + C::NST * C::STAGE;
+    const uint32_t b_empty = b_full + 8 * C::NST;
+    const uint32_t b_done = b_empty + 8 * C::NST;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::NST * C::STAGE + 16 * C::NST + 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * 128, bh = blockIdx.y;
+    const int nchunks = p.T / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(b_full + 8 * s, 1);
+            mbar_init(b_empty + 8 * s, 1);
+        }
+        mbar_init(b_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(smem_addr(tmem_slot), D < 32 ? 32 : D);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (threadIdx.x == 0) {  // producer
+        const uint64_t pol_p = policy_evict_first(), pol_v = policy_evict_last();
+        uint32_t idx = 0, ph = 0;
+        bool ok = true;
+        bool armed[C::NST] = {};
+        uint32_t armed_ph[C::NST] = {};
+        for (int ch = 0; ch < nchunks; ++ch) {
+            if (!mbar_wait(b_empty + 8 * idx, ph ^ 1u, p.limit_ns, W_K3_EMPTY, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint32_t st = base + idx * C::STAGE;
+            mbar_arrive_expect_tx(b_full + 8 * idx, C::STAGE);
+            armed[idx] = true;
+            armed_ph[idx] = ph;
+            tma_load_3d(st, &tmP, b_full + 8 * idx, 64 * ch, m0, bh, pol_p);
+            for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_3d(st + C::P_BYTES + kb * C::V_SUB, &tmV, b_full + 8 * idx, 64 * kb, 64 * ch,
+                            bh, pol_v);
+            if (++idx == (uint32_t)C::NST) { idx = 0; ph ^= 1u; }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            for (int s = 0; s < C::NST; ++s)
+                if (armed[s]) mbar_wait(b_full + 8 * s, armed_ph[s], p.limit_ns, W_K3_FULL);
+        }
+    } else if (threadIdx.x == 32) {  // MMA issuer
+        constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+        uint32_t idx = 0, ph = 0;
+        bool ok = true;
+        for (int ch = 0; ch < nchunks; ++ch) {
+            if (!mbar_wait(b_full + 8 * idx, ph, p.limit_ns, W_K3_FULL, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t st = base + idx * C::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem, sw128_desc(st + kk * 32, 16, 1024),
+                       sw128_desc(st + C::P_BYTES + kk * 2048, C::V_SUB, 1024), idesc,
+                       (ch > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(b_empty + 8 * idx);
+            if (++idx == (uint32_t)C::NST) { idx = 0; ph ^= 1u; }
+        }
+        if (!ok) *abort_flag = 1;
+        tc_commit(b_done);  // fires once every MMA above has completed
+    }
+    __syncwarp();
+    const bool w = mbar_wait(b_done, 0, p.limit_ns, W_K3_DONE);
+    const bool good = __syncthreads_and((w && !*abort_flag) ? 1 : 0) != 0;
+    if (good) {
+        tc_fence_after_sync();
+        const int row = m0 + warp * 32 + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+        __nv_bfloat16 *dst_row = O + ((size_t)bh * p.T + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + 32 * c, r);
+            tmem_wait_ld_regs(r);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst_row + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, D < 32 ? 32 : D);
+}
+
+}  // namespace attn

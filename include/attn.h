@@ -1,0 +1,122 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The operation (per head, Q, K, V each T x d_h):
+ *     O = softmax(mask(scale * Q K^T)) V,   lse_i = log sum_j exp(scale * q_i . k_j)
+ * with the causal mask "key j visible to query i iff j <= i".
+ * Defined in "Why Attention Is Difficult to Optimize" (section "The Attention
+ * Computation Flow": Q, K, V of shape T x d_h, scores divided by sqrt(d_h),
+ * causal mask to -inf, row softmax, O = P V) and in "Attention Mechanism:
+ * Computation & Memory Patterns" (section 1, the three steps S = QK^T,
+ * P = softmax(S / sqrt(d_k)), O = PV).  The fused entry point is the
+ * IO-aware single-kernel form of section 3 of the latter page ("Tiling" +
+ * "Online Softmax"); the unfused entry point is the materialised three-kernel
+ * form of "Storing and Rereading Large Intermediate Matrices".
+ *
+ * Conventions shared by every entry point:
+ *  - Layout: q, k, v, o are bf16, [B, H, T, d_h] contiguous (row = token,
+ *    d_h values contiguous); lse is fp32, [B, H, T].  Head (b, h) starts at
+ *    element ((b * H + h) * T) * d_h.
+ *  - Pointers are device pointers unless the name says host; all must be
+ *    16-byte aligned (tensor-memory-accelerator rule).  The caller owns all
+ *    memory; no entry point allocates device memory.
+ *  - d_h must be 64 or 128.  B, H, T >= 1.  B * H * T must fit in 2^31 - 1
+ *    and T in 2^31 / 256.  scale must be finite and > 0 (configs use
+ *    1 / sqrt(d_h)).  causal is 0 or 1 (top-left aligned, Tq = Tk = T).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The return value reports host-side validation and
+ *    launch errors only; device-side failures (a bounded wait that ran out)
+ *    are read with attn_last_error().
+ *  - Results are deterministic run to run.  The library is thread-compatible,
+ *    not thread-safe: serialise concurrent calls from several host threads.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = 1,           /* a required pointer is NULL                         */
+    ATTN_ERR_UNSUPPORTED_DH = 2, /* d_h not in {64, 128}                               */
+    ATTN_ERR_BAD_SHAPE = 3,      /* B, H or T < 1, or sizes overflow the limits above  */
+    ATTN_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned                   */
+    ATTN_ERR_BAD_SCALE = 5,      /* scale not finite or <= 0                           */
+    ATTN_ERR_LAUNCH = 6,         /* a CUDA runtime/driver call failed                  */
+    ATTN_ERR_TIMEOUT = 7,        /* device: a bounded wait ran out; the kernel returned */
+    ATTN_ERR_NO_DEVICE = 8,      /* no usable sm_100 device is current                 */
+    ATTN_ERR_BAD_ARG = 9         /* another argument is out of range                   */
+} attn_status;
+
+/*
+ * Fused attention forward (one kernel; the T x T score and probability
+ * matrices never reach device memory).
+ *   q, k, v : in,  bf16 [B, H, T, d_h]
+ *   o       : out, bf16 [B, H, T, d_h], each element written once
+ *   lse     : out, fp32 [B, H, T], natural-log log-sum-exp of the scaled,
+ *             masked scores of each query row
+ * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
+             int d_h, int causal, float scale, void *stream);
+
+/*
+ * Unfused attention forward: three kernels with the T x T intermediates in
+ * device memory, as in the materialised path ("Storing and Rereading Large
+ * Intermediate Matrices"):
+ *   K1 writes S = Q K^T (raw, unscaled) to s_ws;
+ *   K2 reads S, scales, masks, applies the row softmax, writes P to p_ws and
+ *      the row log-sum-exp to lse;
+ *   K3 reads P and V and writes O = P V.
+ *   s_ws, p_ws : caller-owned bf16 [B, H, T, T] workspaces (2 bytes per
+ *                entry, the pages' convention), attn_unfused_workspace_bytes()
+ *                bytes each; contents on return are S and P.
+ * T must be a multiple of 128 on this path.  Other arguments as attn_fwd.
+ */
+int attn_fwd_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
+                     void *p_ws, int B, int H, int T, int d_h, int causal, float scale,
+                     void *stream);
+
+/* Bytes of one unfused workspace (S or P): B * H * T * T * 2.  0 on bad sizes. */
+size_t attn_unfused_workspace_bytes(int B, int H, int T);
+
+/*
+ * Fused forward with HOST buffers: copies q/k/v host -> device into the
+ * caller's device buffers dq/dk/dv, runs attn_fwd into do_/dlse, and copies
+ * O and lse back to o_host/lse_host, all in order on `stream`.  Host buffers
+ * should be pinned (cudaHostAlloc) for asynchronous copies.  The call returns
+ * once everything is enqueued; synchronise `stream` before reading o_host.
+ */
+int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                  float *lse_host, void *dq, void *dk, void *dv, void *do_, float *dlse, int B,
+                  int H, int T, int d_h, int causal, float scale, void *stream);
+
+/*
+ * Device status word: synchronises the current device, returns the first
+ * device-side error recorded since the previous call (ATTN_OK if none) and
+ * clears it.  ATTN_ERR_LAUNCH if the synchronisation itself fails.
+ */
+int attn_last_error(void);
+
+/* Static description of a status code. */
+const char *attn_status_str(int status);
+
+/*
+ * Number of SMs the persistent fused kernel sizes its grid by on the current
+ * device (its launch uses min(SMs, work units) CTAs of 320 threads).
+ */
+int attn_fused_grid_ctas(int B, int H, int T, int d_h);
+
+/* Library version, "major.minor.patch". */
+const char *attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,69 @@
+/*
+ * attn_selftest.h -- diagnostic entry points of the B200 attention library.
+ *
+ * These exercise, on one tile, the building blocks the attention kernels are
+ * made of, so that a wrong bit in a descriptor shows up as a wrong number in
+ * a small test rather than inside the full kernel.  They follow the same
+ * conventions as attn.h (device pointers, 16-byte alignment, asynchronous on
+ * `stream`, device errors via attn_last_error()).
+ *
+ * The tile products are the two matrix multiplications of scaled
+ * dot-product attention ("Attention Mechanism: Computation & Memory
+ * Patterns", section 1: S = Q K^T and O = P V), restricted to one 128-row
+ * tile as in the tiled algorithm of section 3 of that page.
+ */
+#ifndef ATTN_B200_SELFTEST_H
+#define ATTN_B200_SELFTEST_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * One score tile on the tensor cores: s[i][j] = sum_c q[i][c] * k[j][c]
+ * for i, j in [0, 128), fp32 accumulation.
+ *   q, k : in,  bf16 [128, d_h] row-major (d_h in {64, 128})
+ *   s    : out, fp32 [128, 128] row-major
+ */
+int attn_selftest_qk_tile(const void *q, const void *k, float *s, int d_h, void *stream);
+
+/*
+ * One output tile with the probabilities held in tensor memory:
+ * o[i][c] = sum_j p[i][j] * v[j][c] for i, j in [0, 128), c in [0, d_h).
+ *   p : in,  bf16 [128, 128] row-major
+ *   v : in,  bf16 [128, d_h] row-major
+ *   o : out, fp32 [128, d_h] row-major
+ */
+int attn_selftest_pv_tile(const void *p, const void *v, float *o, int d_h, void *stream);
+
+/*
+ * Failure detection: launches one CTA that waits on a barrier nothing ever
+ * completes, with a wait limit of `limit_us` microseconds (1 .. 10^6).  The
+ * wait gives up, the kernel records ATTN_ERR_TIMEOUT in the status word and
+ * returns normally, leaving the context usable.  attn_last_error() then
+ * reports ATTN_ERR_TIMEOUT.
+ */
+int attn_selftest_timeout(int limit_us, void *stream);
+
+/*
+ * Scheduling order of the fused kernel's MMA warp.
+ *   mode 0 (default): the next score MMA of a query tile is issued right
+ *     after the PV MMA of that tile, in the tensor core's issue order;
+ *   mode 1: the MMA warp waits for the PV MMA to complete before issuing the
+ *     next score MMA into the same tensor-memory columns.
+ * Both compute the same arithmetic in the same order; the tests compare them
+ * bit for bit.  Returns the previous mode, or -1 for a bad mode.
+ */
+int attn_selftest_set_mma_order(int mode);
+
+/*
+ * Which wait gave up (an internal site code, 0 if none), as read by the most
+ * recent attn_last_error() call; for diagnostics only.
+ */
+int attn_selftest_last_wait_site(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_SELFTEST_H */

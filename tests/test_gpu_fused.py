@@ -1,0 +1,133 @@
+"""Parity of the fused sm_100a forward with the float64 oracle.
+
+Small shapes are compared element by element (every row of every head),
+spanning several tiles and ragged tails; the full-size workloads are compared
+on sampled rows (rows are independent: "Why Attention Is Difficult to
+Optimize", "From a Score Tile to Probabilities" -- scores from other query
+rows are not needed), in the launch configuration the benchmark times."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_124_b200 as attn
+from attn_inputs import WORKLOADS, make_qkv, make_workload, sample_rows
+from tests.gpu_util import check_full, gather, oracle_ref, require_gpu, run_fused, to_dev
+from tests.parity import assert_parity, compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+SWEEP_T = [1, 2, 3, 17, 127, 128, 129, 255, 256, 257, 300, 513]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("T", SWEEP_T)
+def test_tiny_sweep_every_element(T, D, causal):
+    q, k, v = make_qkv(1, 2, T, D, 7000 + T + D + int(causal))
+    st, _ = check_full(q, k, v, causal, 1 / math.sqrt(D))
+    assert_parity(st, f"T={T} D={D} causal={causal}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_multi_head_logit_stress_every_element(D):
+    q, k, v = make_qkv(2, 3, 640, D, 8100 + D, qk_mult=4.0)
+    for causal in (False, True):
+        st, _ = check_full(q, k, v, causal, 1 / math.sqrt(D))
+        assert_parity(st, f"x4 D={D} causal={causal}")
+
+
+def test_tiny_workload_every_element():
+    w = WORKLOADS["tiny_causal_T128_d64"]
+    q, k, v = make_workload(w)
+    st, (o, lse) = check_full(q, k, v, w.causal, w.scale)
+    assert_parity(st, w.name)
+
+
+@pytest.mark.parametrize("name", ["causal_T4096_d64", "causal_T8192_d128",
+                                  "full_T2048_d128_qk4", "causal_T65536_d128"])
+def test_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload(w)
+    o, lse = run_fused(q, k, v, w.causal, w.scale)
+    if w.T >= 65536:
+        heads = [0, w.heads - 1]
+        rows = sample_rows(w.T, w.seed, n_random=96)
+        rows = sorted(set(r for r in rows if r < 256 or r >= w.T - 256 or r % 997 == 0) |
+                      set(sample_rows(w.T, w.seed, n_random=96)[-96:]))
+    else:
+        heads = sorted({0, 1, w.heads // 2, w.heads - 1})
+        rows = sample_rows(w.T, w.seed, n_random=256 if w.T >= 8192 else 512)
+    ro, rl = oracle_ref(q, k, v, w.causal, w.scale, heads=heads, rows=rows)
+    oo, ll = gather(o, lse, heads, rows)
+    st = compare(oo, ll, ro, rl)
+    print(name, st)
+    assert_parity(st, name)
+    # every output finite everywhere, not only at the sampled rows
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def test_causal_row0_is_v0_exactly():
+    q, k, v = make_qkv(2, 4, 1000, 128, 9)
+    o, lse = run_fused(q, k, v, True, 1 / math.sqrt(128))
+    assert torch.equal(o[:, :, 0, :].cpu(), v[:, :, 0, :])
+    ref = (q[:, :, 0, :].double() * k[:, :, 0, :].double()).sum(-1) / math.sqrt(128)
+    assert (lse[:, :, 0].double().cpu() - ref).abs().max().item() < 1e-4
+
+
+def test_deterministic_run_to_run():
+    q, k, v = to_dev(*make_qkv(2, 8, 2048, 128, 11))
+    o1, l1 = attn.fwd(q, k, v, True)
+    o2, l2 = attn.fwd(q, k, v, True)
+    assert attn.last_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("D,causal", [(64, True), (128, True), (128, False)])
+def test_mma_issue_orders_agree_bit_for_bit(D, causal):
+    q, k, v = to_dev(*make_qkv(2, 16, 2048 + 128, D, 12 + D))
+    prev = attn.set_mma_order(1)
+    try:
+        o1, l1 = attn.fwd(q, k, v, causal)
+        assert attn.last_error() == 0
+    finally:
+        attn.set_mma_order(prev)
+    o0, l0 = attn.fwd(q, k, v, causal)
+    assert attn.last_error() == 0
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
+def test_no_quadratic_buffer():
+    w = WORKLOADS["causal_T8192_d128"]
+    q, k, v = to_dev(*make_workload(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    attn.fwd(q, k, v, True, w.scale, o=o, lse=lse)
+    assert attn.last_error() == 0
+    free1, _ = torch.cuda.mem_get_info()
+    # one S for this workload would be 128 heads x 8192^2 x 2 bytes = 16 GiB
+    assert free0 - free1 < (64 << 20)
+
+
+def test_host_buffer_entry_point_matches_device_one():
+    q, k, v = make_qkv(1, 4, 1024, 128, 13)
+    qh, kh, vh = [t.pin_memory() for t in (q, k, v)]
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+    dq, dk, dv = [torch.empty_like(t, device="cuda") for t in (q, k, v)]
+    do_ = torch.empty_like(dq)
+    dl = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    attn.fwd_host(qh, kh, vh, oh, lh, dq, dk, dv, do_, dl, True)
+    torch.cuda.synchronize()
+    assert attn.last_error() == 0
+    o, lse = run_fused(q, k, v, True, 1 / math.sqrt(128))
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
