@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the fused exact-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one fused forward (one kernel launch) over the whole batch of the
+workload, inputs resident in device memory.  The metric is attention-forward
+TFLOP/s, counting 4*T^2*d_h per head and half of that when causal.  Prints ONE
+JSON line (rank 0).
+
+Default workload: B=4, H=32, T=8192, d_h=128, causal (the T >= 8192, d_h = 128
+case the throughput target is quoted on).  Its Q/K/V (3 x 268 MB) are larger
+than the 126 MB L2, so no L2 flush is needed between steps.
+
+Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): heads are
+independent, so every rank runs the whole workload on its own GPU with its own
+seeded inputs and no data-path collective (weak scaling); the only collectives
+are the timing barrier and the max over ranks of the step time.
+
+``--impl reference`` times the float64 CPU oracle (the slow, obviously correct
+program the kernel is checked against) on bounded row samples of the same
+workload, on this host's cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attn_inputs import WORKLOADS, make_qkv, bf16_bits  # noqa: E402
+
+DEFAULT_WORKLOAD = "causal_T8192_d128"
+METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+PEAK_FALLBACK = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_124_b200", "csrc", f)
+                  for f in ("fused_fwd.cuh", "sm100.cuh")]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel from the committed ncu
+    summary, or None when the summary is missing or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", f"fused_fwd_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # pragma: no cover - NVML missing
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def counted_flops(w) -> float:
+    return w.flops()
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, seconds: float, seed_offset: int = 0):
+    """Time the float64 oracle on an evenly spread row sample of head 0 of
+    workload ``w`` sized to about ``seconds`` of CPU work.  Returns
+    (TFLOP/s in the metric's counting, seconds, rows, threads, description)."""
+    import numpy as np
+    import oracle
+    q, k, v = make_qkv(1, 1, w.T, w.D, w.seed + seed_offset, w.qk_mult)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    threads = oracle.default_threads()
+
+    def run(nrows):
+        step = max(1, w.T // nrows)
+        rows = np.arange(step // 2, w.T, step, dtype=np.int64)[:nrows]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qb, kb, vb, w.causal, w.scale, rows=rows, nthreads=threads)
+        dt = time.perf_counter() - t0
+        # the metric's counting: 4*d per visible key (QK^T and PV), per row
+        vis = (rows + 1) if w.causal else np.full(rows.shape, w.T)
+        return rows, dt, float(4.0 * w.D * vis.sum())
+
+    n = max(threads, 32)
+    for _ in range(3):  # calibrate the sample size to the time budget
+        rows, dt, fl = run(n)
+        if dt >= 0.6 * seconds or n >= w.T:
+            break
+        n = int(min(w.T, max(n + 1, n * seconds / max(dt, 1e-6))))
+    desc = (f"{len(rows)} evenly spaced query rows of one head (T={w.T}, d_h={w.D}, "
+            f"{'causal' if w.causal else 'full'}), float64, {threads} threads; FLOPs counted "
+            f"as 4*d_h per visible key")
+    return fl / dt / 1e12, dt, len(rows), threads, desc
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(w, per_step / 4, seed_offset=i)
+    vals, secs = [], []
+    desc, threads = "", 0
+    for i in range(args.steps):
+        v, dt, nrows, threads, desc = oracle_sample(w, per_step, seed_offset=100 + i)
+        vals.append(v)
+        secs.append(dt)
+    value = float(statistics.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.median(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "shape": w.describe(), "seed": w.seed,
+                   "note": "each step times a bounded row sample of the workload"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import exact_attention_124_b200 as attn
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = WORKLOADS[args.workload]
+    attn.load_library()
+    peaks, peak_src = load_peaks()
+
+    # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
+    q, k, v = make_qkv(w.B, w.H, w.T, w.D, w.seed + 1000 * rank, w.qk_mult)
+    dev = torch.device("cuda", local)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.fwd(qd, kd, vd, w.causal, w.scale, o=o, lse=lse, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if attn.last_error() != 0:
+        raise SystemExit("device error during warm-up")
+
+    # timed region: events around every launch on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if world > 1:
+        dist.barrier()
+    status = attn.last_error()
+    launches = args.steps  # one fused kernel per step
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    ms = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = counted_flops(w)
+    value = flops * world / (ms * 1e-3) / 1e12
+    achieved = flops / (statistics.mean(per_launch) * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+
+    # end to end through the host-buffer C-ABI entry point
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.T), dtype=torch.float32).pin_memory()
+    for _ in range(1):
+        attn.fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        attn.fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    status |= attn.last_error()
+    h2d = 3 * q.numel() * 2
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, dt, nrows, threads, desc = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "shape": w.describe(), "global_batch": w.B * world,
+                       "heads": w.H, "seq_len": w.T, "d_h": w.D, "causal": w.causal,
+                       "seed": w.seed, "parallelism": f"heads{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (Q/K/V 3 x %.0f MB); no flush" %
+                             (q.numel() * 2 / 1e6),
+                       "flops_per_step_per_gpu": flops,
+                       "grid_ctas": attn.fused_grid_ctas(w.B, w.H, w.T, w.D, w.causal)},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (cuBLAS bf16 burst)",
+                         "frac_of_sustained": achieved / float(peaks.get(
+                             "bf16_tflops_sustained", peak)),
+                         "frac_of_datasheet_2250": achieved / 2250.0,
+                         "traffic": profiled_traffic(w.name),
+                         "algorithmic_bytes": (3 * q.numel() + o.numel()) * 2 + lse.numel() * 4,
+                         "launch_ms_mean": statistics.mean(per_launch),
+                         "launch_ms_min": min(per_launch)},
+            "clocks": clocks,
+            "gpu_launches": launches,
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "api": "attn_fwd_host"},
+            "cpu_baseline": cpu,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == 0 else 1
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

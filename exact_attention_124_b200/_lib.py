@@ -47,17 +47,18 @@ def load_library():
     lib.attn_last_error.argtypes = []
     lib.attn_status_str.argtypes = [I]
     lib.attn_status_str.restype = ctypes.c_char_p
-    lib.attn_fused_grid_ctas.argtypes = [I, I, I, I]
+    lib.attn_fused_grid_ctas.argtypes = [I, I, I, I, I]
     lib.attn_version.restype = ctypes.c_char_p
     lib.attn_selftest_qk_tile.argtypes = [P, P, P, I, P]
     lib.attn_selftest_pv_tile.argtypes = [P, P, P, I, P]
     lib.attn_selftest_timeout.argtypes = [I, P]
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
+    lib.attn_selftest_set_exp_split.argtypes = [I]
     for name in ("attn_fwd", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
-                 "attn_selftest_last_wait_site"):
+                 "attn_selftest_last_wait_site", "attn_selftest_set_exp_split"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -171,6 +172,19 @@ def set_mma_order(mode: int) -> int:
     if prev < 0:
         raise ValueError("mode must be 0 or 1")
     return prev
+
+
+def set_exp_split(pairs_of_8: int) -> int:
+    """Column pairs out of every 8 whose exponentials run on the FMA pipe
+    (0, 2, 3, 4; -1 = default).  Returns the previous setting."""
+    prev = load_library().attn_selftest_set_exp_split(int(pairs_of_8))
+    if prev == -2:
+        raise ValueError("exp split must be -1, 0, 2, 3 or 4")
+    return prev
+
+
+def fused_grid_ctas(B: int, H: int, T: int, D: int, causal: bool) -> int:
+    return int(load_library().attn_fused_grid_ctas(B, H, T, D, int(bool(causal))))
 
 
 def selftest_qk_tile(q, k, stream=None):

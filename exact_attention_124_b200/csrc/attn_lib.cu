@@ -22,6 +22,8 @@ constexpr int kMaxDevices = 64;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_mma_order = 0;
+int g_exp_split = -1;  // pairs of every 8 on the FMA pipe; -1: per-head-size default
+constexpr int kDefaultSplit64 = 0, kDefaultSplit128 = 0;  // measured fastest on B200
 unsigned int g_last_where = 0;
 
 struct DeviceState {
@@ -52,6 +54,27 @@ bool set_smem(K kernel, int bytes)
            cudaSuccess;
 }
 
+// The fused kernel re-balances registers with setmaxnreg; an increase that
+// the launch's registers cannot cover would wait forever, so refuse to launch
+// a build whose per-thread register count is below the split's assumption.
+template <int D, int EMU>
+bool fused_ready()
+{
+    using C = attn::FusedCfg<D>;
+    if (!set_smem(attn::attn_fwd_fused_kernel<D, EMU>, C::SMEM)) return false;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn::attn_fwd_fused_kernel<D, EMU>) != cudaSuccess)
+        return false;
+    return fa.numRegs >= C::REGS_LAUNCH && fa.maxThreadsPerBlock >= C::THREADS;
+}
+
+template <int D>
+bool fused_all_ready()
+{
+    return fused_ready<D, 0>() && fused_ready<D, 2>() && fused_ready<D, 3>() &&
+           fused_ready<D, 4>();
+}
+
 // Per-device one-time set-up: device check (compute capability 10.0),
 // SM count, shared-memory opt-in of every kernel.
 int device_ready(int *sms_out)
@@ -73,8 +96,8 @@ int device_ready(int *sms_out)
         if (major != 10 || minor != 0 || sms < 1) return ATTN_ERR_NO_DEVICE;
         if (get_encoder() != ATTN_OK) return ATTN_ERR_LAUNCH;
         bool ok = true;
-        ok &= set_smem(attn::attn_fwd_fused_kernel<64>, attn::FusedCfg<64>::SMEM);
-        ok &= set_smem(attn::attn_fwd_fused_kernel<128>, attn::FusedCfg<128>::SMEM);
+        ok &= fused_all_ready<64>();
+        ok &= fused_all_ready<128>();
         ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
         ok &= set_smem(attn::s_gemm_kernel<128>, attn::K1_SMEM);
         ok &= set_smem(attn::pv_gemm_kernel<64>, attn::PvCfg<64>::SMEM);
@@ -134,6 +157,15 @@ int launch_status()
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
+// Persistent grid: one CTA per SM, or fewer when there is less work (causal
+// work is dealt in pairs of query blocks, non-causal in single blocks).
+int fused_grid(long long BH, int T, int causal, int sms)
+{
+    const long long nqb = (T + 255) / 256;
+    const long long work = causal ? BH * ((nqb + 1) / 2) : BH * nqb;
+    return (int)(work < sms ? work : sms);
+}
+
 template <int D>
 int launch_fused(const void *q, const void *k, const void *v, void *o, float *lse, int BH, int T,
                  int causal, float scale, cudaStream_t stream, int sms)
@@ -155,8 +187,14 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     p.nkv = (T + 127) / 128;
     p.order_mode = g_mma_order;
     p.limit_ns = kWaitLimitNs;
-    const int grid = p.units < sms ? p.units : sms;
-    attn::attn_fwd_fused_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    const int grid = fused_grid(BH, T, causal, sms);
+    const int split = g_exp_split >= 0 ? g_exp_split : (D == 64 ? kDefaultSplit64 : kDefaultSplit128);
+    switch (split) {
+        case 0: attn::attn_fwd_fused_kernel<D, 0><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+        case 2: attn::attn_fwd_fused_kernel<D, 2><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+        case 3: attn::attn_fwd_fused_kernel<D, 3><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+        default: attn::attn_fwd_fused_kernel<D, 4><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+    }
     return launch_status();
 }
 
@@ -286,13 +324,12 @@ const char *attn_status_str(int status)
     }
 }
 
-int attn_fused_grid_ctas(int B, int H, int T, int d_h)
+int attn_fused_grid_ctas(int B, int H, int T, int d_h, int causal)
 {
     if (B < 1 || H < 1 || T < 1 || (d_h != 64 && d_h != 128)) return 0;
     int sms = 0;
     if (device_ready(&sms)) return 0;
-    const long long units = (long long)B * H * ((T + 255) / 256);
-    return (int)(units < sms ? units : sms);
+    return fused_grid((long long)B * H, T, causal ? 1 : 0, sms);
 }
 
 const char *attn_version(void) { return "0.1.0"; }
@@ -357,5 +394,15 @@ int attn_selftest_set_mma_order(int mode)
 }
 
 int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
+
+int attn_selftest_set_exp_split(int pairs_of_8)
+{
+    if (pairs_of_8 != -1 && pairs_of_8 != 0 && pairs_of_8 != 2 && pairs_of_8 != 3 &&
+        pairs_of_8 != 4)
+        return -2;
+    const int prev = g_exp_split;
+    g_exp_split = pairs_of_8;
+    return prev;
+}
 
 }  // extern "C"

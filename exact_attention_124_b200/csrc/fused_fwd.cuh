@@ -13,7 +13,7 @@
 // tensor memory (TMEM), P is written back over it as bf16 and read from there
 // by the second MMA.
 //
-// B200 mapping (one persistent CTA per SM, 320 threads):
+// B200 mapping (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for query tile 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax warpgroup for query tile 1 (the two tiles ping-pong, so one
 //              tile's exponentials overlap the other tile's MMAs)
@@ -21,8 +21,12 @@
 //              and O_t += P_t V_j (tmem x smem); allocates/frees TMEM
 //   warp 9     TMA producer (one thread): Q tiles, then K_j / V_j into an
 //              NSTAGE-deep shared-memory ring, in the order the MMA consumes them
-// A work unit is (head, 256 query rows); units are handed out longest-first
-// (causal cost grows with the query block) in a serpentine order over CTAs.
+//   warps 10-11 idle (they complete the third warpgroup, whose registers
+//              setmaxnreg hands to the softmax warpgroups)
+// A work unit is (head, 256 query rows).  Causal: query block q of a head is
+// paired with block nqb-1-q, so every pair costs the same; pairs are dealt
+// round-robin to CTAs in head-major order, so the CTAs running at one time
+// share a few heads' K/V through L2.  Non-causal: units head-major.
 //
 // TMEM (512 columns x 128 lanes x 32 bit):
 //   S_0 / P_0 : columns [0, 128)     S_1 / P_1 : [128, 256)
@@ -39,6 +43,44 @@
 namespace attn {
 
 constexpr float RESCALE_TAU = 8.0f;
+
+// 2^x on the FMA pipe for two values at once (x <= RESCALE_TAU).  Range
+// reduction x = n + f, n = round(x) (adding 1.5 * 2^23 rounds to an integer in
+// the low mantissa bits), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange, computed by gen_exp2_poly.py next to this file; max relative
+// error 7.5e-5, far below the bf16 rounding of P); 2^n by adding n to the
+// exponent field.  x is clamped to -125 first so the result stays a normal
+// number (anything that small is negligible next to the row's terms >= 2^-8).
+constexpr float EXP2_C0 = 0.99992806f;
+constexpr float EXP2_C1 = 0.69326097f;
+constexpr float EXP2_C2 = 0.24261113f;
+constexpr float EXP2_C3 = 0.05517167f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x)
+{
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));   // 1.5 * 2^23 + n
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f)); // n, exactly
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);            // x - n, exactly
+    float2 q = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+    q = __ffma2_rn(q, f, make_float2(EXP2_C1, EXP2_C1));
+    q = __ffma2_rn(q, f, make_float2(EXP2_C0, EXP2_C0));
+    // the low 9 bits of t's pattern hold n (two's complement): shift them into
+    // the exponent field and add
+    const uint32_t ex = __float_as_uint(t.x) << 23, ey = __float_as_uint(t.y) << 23;
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + ex),
+                       __uint_as_float(__float_as_uint(q.y) + ey));
+}
+
+// Which of every 8 consecutive column pairs go to the FMA pipe: the EMU pairs
+// spread evenly over the 8 (EMU = 0 .. 8).
+template <int EMU>
+__device__ __forceinline__ constexpr bool emu_pair(int i)
+{
+    return ((i & 7) * EMU) % 8 + EMU >= 8;
+}
 
 struct FusedParams {
     __nv_bfloat16 *o;
@@ -68,7 +110,15 @@ struct FusedCfg {
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
     static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    // setmaxnreg split: the launch gets 168 registers per thread (384 x 168 =
+    // 64512); the control warpgroup gives back down to 88, the two softmax
+    // warpgroups take 208: 128 x 88 + 256 x 208 = 64512.
+    static constexpr int REGS_LAUNCH = 168;
+    static constexpr int REGS_CTRL = 88;
+    static constexpr int REGS_SOFTMAX = 208;
+    static_assert(128 * REGS_CTRL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH,
+                  "register split exceeds the launch's registers");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_S = 0;            // + 128 * t
     static constexpr uint32_t TM_O = 256;          // + D * t
@@ -87,37 +137,47 @@ struct UnitInfo {
     int niter;
 };
 
-// k-th unit of this CTA in the serpentine, longest-first order; false when
-// the CTA has no k-th unit (callers stop at the first k with k*G >= units and
-// skip the holes of the last round).
-__device__ __forceinline__ bool unit_of(const FusedParams &p, int k, UnitInfo &u)
+// Pairs per head in causal mode (query block q with nqb-1-q).
+__device__ __forceinline__ int pairs_per_head(const FusedParams &p) { return (p.nqb + 1) >> 1; }
+
+// The k-th unit of this CTA.  Returns 1 with `u` filled, 0 for a hole (the
+// middle block of an odd nqb appears once per pair list), -1 when the CTA has
+// no more work.  Every role of the CTA walks the same sequence.
+__device__ __forceinline__ int unit_of(const FusedParams &p, int k, UnitInfo &u)
 {
-    const long long G = gridDim.x;
-    const long long c = blockIdx.x;
-    const long long idx = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
-    if (idx >= p.units) return false;
-    const int level = (int)(idx / p.BH);
-    u.bh = (int)(idx % p.BH);
-    const int qb = p.causal ? (p.nqb - 1 - level) : level;
-    u.i0 = qb * 256;
-    for (int t = 0; t < 2; ++t) {
-        const int r0 = u.i0 + 128 * t;
-        if (r0 >= p.T) {
-            u.n[t] = 0;
-        } else if (p.causal) {
-            const int last = r0 / 128 + 1;
-            u.n[t] = last < p.nkv ? last : p.nkv;
+    const int G = (int)gridDim.x;
+    const int c = (int)blockIdx.x;
+    int qb;
+    if (p.causal) {
+        const int npp = pairs_per_head(p);
+        const int pid = c + G * (k >> 1);   // < BH * npp + G < 2^31 (host-checked sizes)
+        if (pid >= p.BH * npp) return -1;
+        u.bh = pid / npp;
+        const int pp = pid - u.bh * npp;
+        if ((k & 1) == 0) {
+            qb = p.nqb - 1 - pp;
         } else {
-            u.n[t] = p.nkv;
+            qb = pp;
+            if (qb == p.nqb - 1 - pp) return 0;
         }
+    } else {
+        const int pid = c + G * k;
+        if (pid >= p.units) return -1;
+        u.bh = pid / p.nqb;
+        qb = pid - u.bh * p.nqb;
+    }
+    u.i0 = qb * 256;
+    const int r1 = u.i0 + 128;
+    if (p.causal) {
+        const int l0 = r1 / 128;           // = i0/128 + 1
+        u.n[0] = l0 < p.nkv ? l0 : p.nkv;
+        u.n[1] = r1 >= p.T ? 0 : (l0 + 1 < p.nkv ? l0 + 1 : p.nkv);
+    } else {
+        u.n[0] = p.nkv;
+        u.n[1] = r1 >= p.T ? 0 : p.nkv;
     }
     u.niter = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
-    return true;
-}
-
-__device__ __forceinline__ bool more_units(const FusedParams &p, int k)
-{
-    return (long long)k * gridDim.x < p.units;
+    return 1;
 }
 
 struct Ring {
@@ -132,8 +192,8 @@ struct Ring {
     }
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+template <int D, int EMU>
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const FusedParams p)
@@ -195,7 +255,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tmem = *tmem_slot;
     const uint64_t lim = p.limit_ns;
 
-    if (warp == 9) {
+    if (warp >= 8) {
+      reg_dealloc<C::REGS_CTRL>();
+      if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = policy_evict_first();
@@ -218,9 +280,11 @@ __global__ void __launch_bounds__(320, 1)
                 ring.advance<C::NSTAGE>();
                 return true;
             };
-            for (int k = 0; ok && more_units(p, k); ++k) {
+            for (int k = 0; ok; ++k) {
                 UnitInfo u;
-                if (!unit_of(p, k, u)) continue;
+                const int r = unit_of(p, k, u);
+                if (r < 0) break;
+                if (r == 0) continue;
                 if (*abort_flag) { ok = false; break; }
                 #pragma unroll
                 for (int t = 0; t < 2 && ok; ++t) {
@@ -254,7 +318,7 @@ __global__ void __launch_bounds__(320, 1)
                         mbar_wait(b_qfull + 8 * t, (q_armed_par >> t) & 1u, lim, W_QFULL);
             }
         }
-    } else if (warp == 8) {
+      } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             Ring ring;
@@ -272,28 +336,31 @@ __global__ void __launch_bounds__(320, 1)
                 drain_ph ^= 1u;
                 return r;
             };
+            // descriptor low words advance by (byte offset >> 4); high words are fixed
             auto qk = [&](int t, uint32_t kslot) {
-                const uint32_t qa = sQ + t * C::TILE;
-                const uint32_t kbse = sKV + kslot * C::TILE;
+                const uint32_t qa = sw128_desc_lo(sQ + t * C::TILE, 16);
+                const uint32_t ka = sw128_desc_lo(sKV + kslot * C::TILE, 16);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::SUB + (kk & 3) * 32;
-                    mma_ss(tS[t], sw128_desc(qa + off, 16, 1024), sw128_desc(kbse + off, 16, 1024),
+                    const uint32_t off = ((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4;
+                    mma_ss(tS[t], sw128_desc_join(qa + off, 1024), sw128_desc_join(ka + off, 1024),
                            C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
             };
             auto pv = [&](int t, uint32_t vslot, bool acc) {
-                const uint32_t vb = sKV + vslot * C::TILE;
+                const uint32_t va = sw128_desc_lo(sKV + vslot * C::TILE, C::SUB);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tO[t], tS[t] + 8 * kk, sw128_desc(vb + kk * 2048, C::SUB, 1024),
+                    mma_ts(tO[t], tS[t] + 8 * kk, sw128_desc_join(va + kk * (2048 >> 4), 1024),
                            C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
             };
 
-            for (int k = 0; ok && more_units(p, k); ++k) {
+            for (int k = 0; ok; ++k) {
                 UnitInfo u;
-                if (!unit_of(p, k, u)) continue;
-                #pragma unroll
+                const int r = unit_of(p, k, u);
+                if (r < 0) break;
+                if (r == 0) continue;
+#pragma unroll
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (u.n[t] == 0) continue;
                     ok = mbar_wait(b_qfull + 8 * t, qph[t], lim, W_QFULL, abort_flag);
@@ -367,8 +434,10 @@ __global__ void __launch_bounds__(320, 1)
                 drain();  // every issued MMA finishes before TMEM is freed
             }
         }
+      }
     } else {
         // ------------------------------------------------------------ softmax warpgroups
+        reg_alloc<C::REGS_SOFTMAX>();
         const int t = warp >> 2;          // query tile 0 or 1
         const int wq = warp & 3;          // TMEM lane quarter
         const int rit = wq * 32 + lane;   // row in tile == TMEM lane
@@ -378,9 +447,11 @@ __global__ void __launch_bounds__(320, 1)
         const float cl2 = p.c_log2;
         uint32_t sph = 0, oph = 0;
         bool ok = true;
-        for (int k = 0; ok && more_units(p, k); ++k) {
+        for (int k = 0; ok; ++k) {
             UnitInfo u;
-            if (!unit_of(p, k, u)) continue;
+            const int r = unit_of(p, k, u);
+            if (r < 0) break;
+            if (r == 0) continue;
             const int nt = u.n[t];
             if (nt == 0) continue;
             const int r0 = u.i0 + 128 * t;
@@ -410,13 +481,18 @@ __global__ void __launch_bounds__(320, 1)
                     for (int c = 0; c < 128; ++c)
                         if (key0 + c > lim_key) s[c] = -INFINITY;
                 }
-                float mx[8];
+                // row maximum: four running maxima, two new columns each per step
+                float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = s[i];
-#pragma unroll
-                for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-                const float rowmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int c = 4; c + 8 <= 128; c += 8) {  // columns 4 .. 123
+                    mx[0] = max3(mx[0], s[c], s[c + 1]);
+                    mx[1] = max3(mx[1], s[c + 2], s[c + 3]);
+                    mx[2] = max3(mx[2], s[c + 4], s[c + 5]);
+                    mx[3] = max3(mx[3], s[c + 6], s[c + 7]);
+                }
+                mx[0] = max3(mx[0], s[124], s[125]);
+                mx[1] = max3(mx[1], s[126], s[127]);
+                const float rowmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]);
                 const float cand = rowmax * cl2;
                 float alpha = 1.f;
                 bool resc = false;
@@ -441,21 +517,50 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 l *= alpha;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                const float2 c2 = make_float2(cl2, cl2);
+                const float2 nm2 = make_float2(neg_m, neg_m);
+                float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                // p = 2^(s * scale * log2e - m); on tiles without masked keys a
+                // fixed share of the pairs (EMU of every 8) is evaluated on the
+                // FMA pipe, the rest by MUFU.EX2, so the two pipes share the load.
+                if (EMU > 0 && !need_mask) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[32];
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float p0 = fast_exp2(fmaf(s[64 * h + 2 * i], cl2, neg_m));
-                        const float p1 = fast_exp2(fmaf(s[64 * h + 2 * i + 1], cl2, neg_m));
-                        ls[(2 * i) & 3] += p0;
-                        ls[(2 * i + 1) & 3] += p1;
-                        pk[i] = pack_bf16x2(p0, p1);
+                        for (int i = 0; i < 32; ++i) {
+                            const float2 x = __ffma2_rn(
+                                make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
+                            float2 pr;
+                            if (emu_pair<EMU>(i)) {
+                                pr = exp2_poly2(x);
+                            } else {
+                                pr.x = fast_exp2(x.x);
+                                pr.y = fast_exp2(x.y);
+                            }
+                            ls[i & 1] = __fadd2_rn(ls[i & 1], pr);
+                            pk[i] = pack_bf16x2(pr.x, pr.y);
+                        }
+                        tmem_st32(tS + 32 * h, pk);
                     }
-                    tmem_st32(tS + 32 * h, pk);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float2 x = __ffma2_rn(
+                                make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
+                            float2 pr;
+                            pr.x = fast_exp2(x.x);
+                            pr.y = fast_exp2(x.y);
+                            ls[i & 1] = __fadd2_rn(ls[i & 1], pr);
+                            pk[i] = pack_bf16x2(pr.x, pr.y);
+                        }
+                        tmem_st32(tS + 32 * h, pk);
+                    }
                 }
-                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
                 tmem_wait_st();
                 tc_fence_before_sync();
                 mbar_arrive(b_pfull + 8 * t);

@@ -277,6 +277,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
     return d;
 }
 
+// The same descriptor split in two 32-bit words: the low word carries the
+// start address and the leading byte offset, so moving along a buffer only
+// adds (bytes >> 4) to it (addresses stay below 2^18, no carry into bit 14).
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo_bytes)
+{
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+
+__device__ __forceinline__ uint64_t sw128_desc_join(uint32_t lo, uint32_t sbo_bytes)
+{
+    const uint32_t hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+    return ((uint64_t)hi << 32) | lo;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B and an fp32 accumulator:
 //   bits 4-5 D format (1 = f32)   bits 7-9 A format (1 = bf16)
 //   bits 10-12 B format (1 = bf16)  bit 15 A major (0 = K)  bit 16 B major
@@ -285,6 +299,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Register re-balancing between warpgroups (all four warps of a warpgroup
+// execute it).  The increase waits until the decreases of other warpgroups
+// have returned enough registers, so the split must fit the launch's total.
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -107,10 +107,12 @@ int attn_last_error(void);
 const char *attn_status_str(int status);
 
 /*
- * Number of SMs the persistent fused kernel sizes its grid by on the current
- * device (its launch uses min(SMs, work units) CTAs of 320 threads).
+ * CTAs the persistent fused kernel launches for this problem on the current
+ * device: min(SMs, work items) CTAs of 384 threads, where a work item is a
+ * block of 256 query rows of one head (causal: a pair of such blocks).
+ * 0 on bad sizes or without a device.
  */
-int attn_fused_grid_ctas(int B, int H, int T, int d_h);
+int attn_fused_grid_ctas(int B, int H, int T, int d_h, int causal);
 
 /* Library version, "major.minor.patch". */
 const char *attn_version(void);

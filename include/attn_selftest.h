@@ -57,6 +57,15 @@ int attn_selftest_timeout(int limit_us, void *stream);
 int attn_selftest_set_mma_order(int mode);
 
 /*
+ * Share of the softmax exponentials evaluated on the FMA pipe instead of the
+ * special-function unit, in column pairs out of every 8: 0, 2, 3 or 4; -1
+ * restores the per-head-size default.  Only tiles without masked keys use
+ * the FMA-pipe form; results differ from the all-MUFU form by rounding only.
+ * Returns the previous setting, or -2 for a value not built.
+ */
+int attn_selftest_set_exp_split(int pairs_of_8);
+
+/*
  * Which wait gave up (an internal site code, 0 if none), as read by the most
  * recent attn_last_error() call; for diagnostics only.
  */

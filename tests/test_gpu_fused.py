@@ -131,3 +131,17 @@ def test_host_buffer_entry_point_matches_device_one():
     assert attn.last_error() == 0
     o, lse = run_fused(q, k, v, True, 1 / math.sqrt(128))
     assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
+
+
+@pytest.mark.parametrize("split", [0, 2, 3, 4])
+@pytest.mark.parametrize("D", [64, 128])
+def test_every_exp_split_every_element(split, D):
+    """Each share of FMA-pipe exponentials meets the same parity bar."""
+    q, k, v = make_qkv(2, 2, 1024 + 64, D, 9100 + D + split, qk_mult=2.0)
+    prev = attn.set_exp_split(split)
+    try:
+        for causal in (True, False):
+            st, _ = check_full(q, k, v, causal, 1 / math.sqrt(D))
+            assert_parity(st, f"split={split} D={D} causal={causal}")
+    finally:
+        attn.set_exp_split(prev)
