@@ -320,6 +320,7 @@ const char *attn_status_str(int status)
         case ATTN_ERR_TIMEOUT: return "device wait timed out";
         case ATTN_ERR_NO_DEVICE: return "no sm_100 device";
         case ATTN_ERR_BAD_ARG: return "bad argument";
+        case ATTN_ERR_WORKSPACE_LIMIT: return "problem exceeds the static workspace (B*H*T*T > 16777216)";
         default: return "unknown status";
     }
 }
@@ -406,3 +407,50 @@ int attn_selftest_set_exp_split(int pairs_of_8)
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ allocation-free unfused forward
+// Callers that cannot allocate device memory (a plug-in whose host owns the
+// device through its own memory pool, or code that must not risk the
+// synchronisation an allocation or free can cause) get S and P from this
+// static array instead of caller-provided workspaces: 64 MiB, S in the first
+// half and P in the second.  Every GPU that loads the library reserves it
+// until the process exits.  In host code the symbol is only a host-side
+// stand-in; its device address is looked up per device (below) and passed to
+// the kernels.
+constexpr size_t kNoallocBytes = (size_t)64 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_ws[kNoallocBytes];
+
+namespace {
+void *g_noalloc_dev_ptr[kMaxDevices] = {};
+}
+
+extern "C" int attn_fwd_unfused_noalloc(const void *q, const void *k, const void *v, void *o,
+                                        float *lse, int B, int H, int T, int d_h, int causal,
+                                        float scale, void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    if (T % 128 != 0 || (long long)B * H > 65535) return ATTN_ERR_BAD_SHAPE;
+    const unsigned long long one = (unsigned long long)B * H * T * (unsigned long long)T * 2ull;
+    if (one > kNoallocBytes / 2) return ATTN_ERR_WORKSPACE_LIMIT;
+    if ((rc = device_ready(nullptr))) return rc;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        (void)cudaGetLastError();
+        return ATTN_ERR_NO_DEVICE;
+    }
+    if (g_noalloc_dev_ptr[dev] == nullptr) {  // first call on this device
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_ws) != cudaSuccess || ptr == nullptr) {
+            (void)cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        g_noalloc_dev_ptr[dev] = ptr;
+    }
+    auto *ws = static_cast<unsigned char *>(g_noalloc_dev_ptr[dev]);
+    void *s_ws = ws;
+    void *p_ws = ws + kNoallocBytes / 2;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s)
+                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s);
+}

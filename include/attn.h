@@ -50,7 +50,8 @@ typedef enum {
     ATTN_ERR_LAUNCH = 6,         /* a CUDA runtime/driver call failed                  */
     ATTN_ERR_TIMEOUT = 7,        /* device: a bounded wait ran out; the kernel returned */
     ATTN_ERR_NO_DEVICE = 8,      /* no usable sm_100 device is current                 */
-    ATTN_ERR_BAD_ARG = 9         /* another argument is out of range                   */
+    ATTN_ERR_BAD_ARG = 9,        /* another argument is out of range                   */
+    ATTN_ERR_WORKSPACE_LIMIT = 10 /* problem too large for the library's static workspace */
 } attn_status;
 
 /*
@@ -84,6 +85,29 @@ int attn_fwd_unfused(const void *q, const void *k, const void *v, void *o, float
 
 /* Bytes of one unfused workspace (S or P): B * H * T * T * 2.  0 on bad sizes. */
 size_t attn_unfused_workspace_bytes(int B, int H, int T);
+
+/*
+ * Unfused forward that allocates nothing and takes no workspace: S and P live
+ * in a static device array inside the library (64 MiB, 32 MiB each for S and
+ * P, reserved on every GPU that loads the library until the process exits).
+ * The pages have no counterpart; this entry point exists for callers that
+ * cannot call cudaMalloc -- for instance a plug-in inside a host application
+ * that owns all device memory through its own pool, where a foreign
+ * allocation can fail or break the host's accounting, or code that must not
+ * risk the device synchronisation an allocation or free can cause.
+ *   Sizes: as attn_fwd_unfused, plus B * H * T * T <= 16,777,216 (for
+ *   example one head at T = 4096, or 16 heads at T = 1024); larger problems
+ *   return ATTN_ERR_WORKSPACE_LIMIT and launch nothing.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) for that device; make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one array and leaves its S and P there;
+ *   nothing in it needs to start at zero (each call writes all of S and P
+ *   before reading them).  Calls whose work overlaps on the GPU (several
+ *   streams, or several host threads) race on the array: serialise them.
+ */
+int attn_fwd_unfused_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                             int B, int H, int T, int d_h, int causal, float scale, void *stream);
 
 /*
  * Fused forward with HOST buffers: copies q/k/v host -> device into the
