@@ -164,6 +164,29 @@ def counted_flops(w) -> float:
     return w.flops()
 
 
+def rank_seed(w, rank: int) -> int:
+    """Each rank draws its own inputs: the workload's seed offset by 1000 * rank."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of ``x`` over all ranks (the slowest rank sets the step
+    time); a plain return when running alone."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank does flops_per_rank per step; the job's step
+    takes the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------------- CPU oracle
 def oracle_sample(w, seconds: float, seed_offset: int = 0):
     """Time the float64 oracle on an evenly spread row sample of head 0 of
@@ -246,7 +269,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
 
     # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
-    q, k, v = make_qkv(w.B, w.H, w.T, w.D, w.seed + 1000 * rank, w.qk_mult)
+    q, k, v = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)
     dev = torch.device("cuda", local)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     o = torch.empty_like(qd)
@@ -280,13 +303,9 @@ def run_ours(args):
     launches = args.steps  # one fused kernel per step
     per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
-    ms = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(total_ms / args.steps, world, dev)
     flops = counted_flops(w)
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms)
     achieved = flops / (statistics.mean(per_launch) * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
 
@@ -306,11 +325,7 @@ def run_ours(args):
         attn.fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
     status |= attn.last_error()
     h2d = 3 * q.numel() * 2
     d2h = o.numel() * 2 + lse.numel() * 4
@@ -348,7 +363,7 @@ def run_ours(args):
                          "launch_ms_min": min(per_launch)},
             "clocks": clocks,
             "gpu_launches": launches,
-            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "api": "attn_fwd_host"},
             "cpu_baseline": cpu,
