@@ -58,7 +58,21 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["fused", "unfused"], default="fused",
+                    help="unfused: the three-kernel materialised path (S and P in HBM)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's B")
+    ap.add_argument("--exp-split", type=int, default=None,
+                    help="fused kernel variant: column pairs of every 8 whose exponentials run "
+                         "on the FMA pipe (0, 2, 3, 4); default: the library's choice")
     return ap.parse_args()
+
+
+def workload_of(args):
+    import dataclasses
+    w = WORKLOADS[args.workload]
+    if args.batch:
+        w = dataclasses.replace(w, B=int(args.batch), name=f"{w.name}_B{int(args.batch)}")
+    return w
 
 
 def load_peaks():
@@ -224,7 +238,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_sample(w, per_step / 4, seed_offset=i)
@@ -264,9 +278,13 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     attn.load_library()
+    if args.exp_split is not None:
+        attn.set_exp_split(args.exp_split)
     peaks, peak_src = load_peaks()
+    if args.path == "unfused":
+        return run_unfused(args, w, world, rank, local, peaks, peak_src)
 
     # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
     q, k, v = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)
@@ -373,6 +391,66 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0 if status == 0 else 1
+
+
+def unfused_bytes(w) -> int:
+    """Algorithmic HBM bytes of the materialised path per step: S written and
+    read, P written and read (bf16, T^2 per head each), plus Q, K, V read (K1
+    reads Q and K, K3 reads V), O written (bf16) and lse written (fp32)."""
+    heads = w.B * w.H
+    return heads * (4 * w.T * w.T * 2 + 4 * w.T * w.D * 2 + w.T * 4)
+
+
+def run_unfused(args, w, world, rank, local, peaks, peak_src):
+    import torch
+    import exact_attention_124_b200 as attn
+    dev = torch.device("cuda", local)
+    q, k, v = [t.to(dev) for t in make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)]
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+    S = torch.empty((w.B, w.H, w.T, w.T), dtype=torch.bfloat16, device=dev)
+    P = torch.empty_like(S)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.fwd_unfused(q, k, v, w.causal, w.scale, o=o, lse=lse, s_ws=S, p_ws=P, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if attn.last_error() != 0:
+        raise SystemExit("device error during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    status = attn.last_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    nbytes = unfused_bytes(w)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    if rank == 0:
+        line = {
+            "metric": METRIC + " (unfused three-kernel path)", "path": "unfused",
+            "value": whole_job_tflops(counted_flops(w), world, ms), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "shape": w.describe(), "seed": w.seed,
+                       "workspace_bytes": 2 * S.numel() * 2},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic_bytes": nbytes, "traffic": None},
+            "clocks": sampler.summary(), "gpu_launches": 3 * args.steps,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
     return 0 if status == 0 else 1
 
 

@@ -108,7 +108,7 @@ struct FusedCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+    static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 4 + 2 + 1;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
     static constexpr int THREADS = 384;
     // setmaxnreg split: the launch gets 168 registers per thread (384 x 168 =
@@ -130,6 +130,45 @@ struct FusedCfg {
 enum : unsigned int {
     W_QFULL = 1, W_QEMPTY, W_KVFULL, W_KVEMPTY, W_SFULL, W_PFULL, W_PVDONE, W_DRAIN
 };
+
+// Row maximum of 128 scores: eight independent running maxima (two new
+// columns each per step), then a short tree.
+__device__ __forceinline__ float row_max(const float (&s)[128])
+{
+    float mx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+    for (int c = 8; c < 120; c += 16) {  // columns 8 .. 119
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx[i] = max3(mx[i], s[120 + 2 * i], s[121 + 2 * i]);
+    return max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
+// p = 2^(s * c - m) for column pairs P0 .. P0+NP-1, packed to bf16 pairs in pk;
+// the fp32 p are summed into ls (two packed accumulators).
+template <int EMU, int P0, int NP>
+__device__ __forceinline__ void exp_pairs(const float (&s)[128], float2 c2, float2 nm2,
+                                          uint32_t (&pk)[NP], float2 (&ls)[2])
+{
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+        const int pi = P0 + i;
+        const float2 x = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), c2, nm2);
+        float2 pr;
+        if (emu_pair<EMU>(pi)) {
+            pr = exp2_poly2(x);
+        } else {
+            pr.x = fast_exp2(x.x);
+            pr.y = fast_exp2(x.y);
+        }
+        ls[i & 1] = __fadd2_rn(ls[i & 1], pr);
+        pk[i] = pack_bf16x2(pr.x, pr.y);
+    }
+}
 
 struct UnitInfo {
     int bh, i0;
@@ -213,8 +252,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t b_kvfull = bar0 + 32;                    // [NSTAGE]
     const uint32_t b_kvempty = b_kvfull + 8 * C::NSTAGE;    // [NSTAGE]
     const uint32_t b_sfull = b_kvempty + 8 * C::NSTAGE;     // [2]
-    const uint32_t b_pfull = b_sfull + 16;                  // [2]
-    const uint32_t b_pvdone = b_pfull + 16;                 // [2]
+    const uint32_t b_pfull = b_sfull + 16;                  // [2 tiles][2 halves]
+    const uint32_t b_pvdone = b_pfull + 32;                 // [2]
     const uint32_t b_drain = b_pvdone + 16;                 // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -233,7 +272,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(b_sfull + 8 * t, 1);
-            mbar_init(b_pfull + 8 * t, 128);
+            mbar_init(b_pfull + 16 * t, 128);      // keys 0-63 of P_t written
+            mbar_init(b_pfull + 16 * t + 8, 128);  // keys 64-127 of P_t written
             mbar_init(b_pvdone + 8 * t, 1);
         }
         mbar_init(b_drain, 1);
@@ -347,12 +387,23 @@ __global__ void __launch_bounds__(384, 1)
                            C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
             };
-            auto pv = [&](int t, uint32_t vslot, bool acc) {
+            // O_t (+)= P_t V: each half of P (64 keys) is consumed as soon as the
+            // softmax warpgroup has written it, so the first half of the MMA
+            // overlaps the exponentials of the second half.
+            auto pv = [&](int t, uint32_t vslot, bool acc) -> bool {
                 const uint32_t va = sw128_desc_lo(sKV + vslot * C::TILE, C::SUB);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tO[t], tS[t] + 8 * kk, sw128_desc_join(va + kk * (2048 >> 4), 1024),
-                           C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < 2; ++h) {
+                    if (!mbar_wait(b_pfull + 16 * t + 8 * h, pph[t], lim, W_PFULL, abort_flag))
+                        return false;
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+                        mma_ts(tO[t], tS[t] + 8 * kk, sw128_desc_join(va + kk * (2048 >> 4), 1024),
+                               C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                }
+                pph[t] ^= 1u;
+                return true;
             };
 
             for (int k = 0; ok; ++k) {
@@ -394,10 +445,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         if (j - 1 < u.n[t]) {  // O_t += P_t(j-1) V_{j-1}
-                            if (!(ok = mbar_wait(b_pfull + 8 * t, pph[t], lim, W_PFULL, abort_flag))) break;
-                            pph[t] ^= 1u;
-                            tc_fence_after_sync();
-                            pv(t, vs, j - 1 > 0);
+                            if (!(ok = pv(t, vs, j - 1 > 0))) break;
                             if (j - 1 == u.n[t] - 1) tc_commit(b_pvdone + 8 * t);
                         }
                         if (j < u.n[t]) {      // S_t = Q_t K_j^T
@@ -419,10 +467,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (u.niter - 1 < u.n[t]) {
-                        if (!(ok = mbar_wait(b_pfull + 8 * t, pph[t], lim, W_PFULL, abort_flag))) break;
-                        pph[t] ^= 1u;
-                        tc_fence_after_sync();
-                        pv(t, vs, u.niter - 1 > 0);
+                        if (!(ok = pv(t, vs, u.niter - 1 > 0))) break;
                         tc_commit(b_pvdone + 8 * t);
                     }
                 }
@@ -465,13 +510,12 @@ __global__ void __launch_bounds__(384, 1)
                 sph ^= 1u;
                 tc_fence_after_sync();
                 float s[128];
+                {
+                    uint32_t r[128];
+                    tmem_ld128(tS, r);
+                    tmem_wait_ld_regs128(r);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + 32 * c, r);
-                    tmem_wait_ld_regs(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i]);
                 }
                 const int key0 = 128 * j;
                 const bool need_mask = (p.causal && key0 + 127 > r0) || (key0 + 128 > p.T);
@@ -481,19 +525,7 @@ __global__ void __launch_bounds__(384, 1)
                     for (int c = 0; c < 128; ++c)
                         if (key0 + c > lim_key) s[c] = -INFINITY;
                 }
-                // row maximum: four running maxima, two new columns each per step
-                float mx[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-                for (int c = 4; c + 8 <= 128; c += 8) {  // columns 4 .. 123
-                    mx[0] = max3(mx[0], s[c], s[c + 1]);
-                    mx[1] = max3(mx[1], s[c + 2], s[c + 3]);
-                    mx[2] = max3(mx[2], s[c + 4], s[c + 5]);
-                    mx[3] = max3(mx[3], s[c + 6], s[c + 7]);
-                }
-                mx[0] = max3(mx[0], s[124], s[125]);
-                mx[1] = max3(mx[1], s[126], s[127]);
-                const float rowmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]);
-                const float cand = rowmax * cl2;
+                const float cand = row_max(s) * cl2;
                 float alpha = 1.f;
                 bool resc = false;
                 if (j == 0) {
@@ -518,52 +550,29 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const float2 c2 = make_float2(cl2, cl2);
-                const float2 nm2 = make_float2(neg_m, neg_m);
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                // p = 2^(s * scale * log2e - m); on tiles without masked keys a
+                // p = 2^(s * scale * log2e - m).  On tiles without masked keys a
                 // fixed share of the pairs (EMU of every 8) is evaluated on the
-                // FMA pipe, the rest by MUFU.EX2, so the two pipes share the load.
-                if (EMU > 0 && !need_mask) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float2 x = __ffma2_rn(
-                                make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
-                            float2 pr;
-                            if (emu_pair<EMU>(i)) {
-                                pr = exp2_poly2(x);
-                            } else {
-                                pr.x = fast_exp2(x.x);
-                                pr.y = fast_exp2(x.y);
-                            }
-                            ls[i & 1] = __fadd2_rn(ls[i & 1], pr);
-                            pk[i] = pack_bf16x2(pr.x, pr.y);
-                        }
-                        tmem_st32(tS + 32 * h, pk);
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float2 x = __ffma2_rn(
-                                make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
-                            float2 pr;
-                            pr.x = fast_exp2(x.x);
-                            pr.y = fast_exp2(x.y);
-                            ls[i & 1] = __fadd2_rn(ls[i & 1], pr);
-                            pk[i] = pack_bf16x2(pr.x, pr.y);
-                        }
-                        tmem_st32(tS + 32 * h, pk);
-                    }
-                }
-                l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+                // FMA pipe, the rest by MUFU.EX2.
+                uint32_t pk0[32];
+                if (EMU > 0 && !need_mask)
+                    exp_pairs<EMU, 0, 32>(s, c2, make_float2(neg_m, neg_m), pk0, ls);
+                else
+                    exp_pairs<0, 0, 32>(s, c2, make_float2(neg_m, neg_m), pk0, ls);
+                tmem_st32(tS, pk0);
                 tmem_wait_st();
                 tc_fence_before_sync();
-                mbar_arrive(b_pfull + 8 * t);
+                mbar_arrive(b_pfull + 16 * t);  // keys 0-63 of P are in TMEM
+                uint32_t pk1[32];
+                if (EMU > 0 && !need_mask)
+                    exp_pairs<EMU, 32, 32>(s, c2, make_float2(neg_m, neg_m), pk1, ls);
+                else
+                    exp_pairs<0, 32, 32>(s, c2, make_float2(neg_m, neg_m), pk1, ls);
+                tmem_st32(tS + 32, pk1);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(b_pfull + 16 * t + 8);  // keys 64-127
+                l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
             }
             if (!ok) break;
             // epilogue: O = acc / l, lse = (m + log2 l) ln 2
