@@ -40,6 +40,7 @@ def load_library():
     lib = ctypes.CDLL(_SO)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.attn_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_fwd_unfused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_unfused_workspace_bytes.argtypes = [I, I, I]
@@ -55,7 +56,7 @@ def load_library():
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
-    for name in ("attn_fwd", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
+    for name in ("attn_fwd", "attn_fwd_gqa", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
                  "attn_selftest_last_wait_site", "attn_selftest_set_exp_split"):
@@ -113,6 +114,28 @@ def fwd(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, str
     rc = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                       B, H, T, D, int(bool(causal)), float(scale), _stream(stream))
     _check(rc, "attn_fwd")
+    return o, lse
+
+
+def fwd_gqa(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, stream=None):
+    """Fused forward with grouped-query attention: q [B, H, T, d_h], k and v
+    [B, H_kv, T, d_h] with H % H_kv == 0.  Returns (o, lse)."""
+    lib = load_library()
+    B, H, T, D = _shape(q)
+    Bk, H_kv, Tk, Dk = _shape(k)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t, n)
+    if (Bk, Tk, Dk) != (B, T, D) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k/v must be [B, H_kv, T, d_h] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    rc = lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, H, H_kv, T, D, int(bool(causal)), float(scale), _stream(stream))
+    _check(rc, "attn_fwd_gqa")
     return o, lse
 
 

@@ -167,18 +167,21 @@ int fused_grid(long long BH, int T, int causal, int sms)
 }
 
 template <int D>
-int launch_fused(const void *q, const void *k, const void *v, void *o, float *lse, int BH, int T,
-                 int causal, float scale, cudaStream_t stream, int sms)
+int launch_fused(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                 int H_kv, int T, int causal, float scale, cudaStream_t stream, int sms)
 {
     using C = attn::FusedCfg<D>;
+    const int BH = B * H;
     CUtensorMap mq, mk, mv;
-    if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, BH, 128) ||
-        make_map(&mv, v, D, T, BH, 128))
+    if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, (uint64_t)B * H_kv, 128) ||
+        make_map(&mv, v, D, T, (uint64_t)B * H_kv, 128))
         return ATTN_ERR_LAUNCH;
     attn::FusedParams p;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.BH = BH;
+    p.H = H;
+    p.group = H / H_kv;
     p.T = T;
     p.causal = causal;
     p.c_log2 = scale * 1.4426950408889634f;
@@ -237,8 +240,21 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
     int sms = 0;
     if ((rc = device_ready(&sms))) return rc;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return d_h == 64 ? launch_fused<64>(q, k, v, o, lse, B * H, T, causal, scale, s, sms)
-                     : launch_fused<128>(q, k, v, o, lse, B * H, T, causal, scale, s, sms);
+    return d_h == 64 ? launch_fused<64>(q, k, v, o, lse, B, H, H, T, causal, scale, s, sms)
+                     : launch_fused<128>(q, k, v, o, lse, B, H, H, T, causal, scale, s, sms);
+}
+
+int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                 int H_kv, int T, int d_h, int causal, float scale, void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    if (H_kv < 1 || H % H_kv != 0) return ATTN_ERR_BAD_SHAPE;
+    int sms = 0;
+    if ((rc = device_ready(&sms))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64 ? launch_fused<64>(q, k, v, o, lse, B, H, H_kv, T, causal, scale, s, sms)
+                     : launch_fused<128>(q, k, v, o, lse, B, H, H_kv, T, causal, scale, s, sms);
 }
 
 size_t attn_unfused_workspace_bytes(int B, int H, int T)

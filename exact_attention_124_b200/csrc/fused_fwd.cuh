@@ -27,6 +27,9 @@
 // paired with block nqb-1-q, so every pair costs the same; pairs are dealt
 // round-robin to CTAs in head-major order, so the CTAs running at one time
 // share a few heads' K/V through L2.  Non-causal: units head-major.
+// Grouped-query attention: query head h of batch entry b reads K/V head
+// b * (H / group) + h / group; the head-major order keeps a group's query
+// heads on neighbouring CTAs, which then share that K/V head through L2.
 //
 // TMEM (512 columns x 128 lanes x 32 bit):
 //   S_0 / P_0 : columns [0, 128)     S_1 / P_1 : [128, 256)
@@ -85,7 +88,9 @@ __device__ __forceinline__ constexpr bool emu_pair(int i)
 struct FusedParams {
     __nv_bfloat16 *o;
     float *lse;
-    int BH;
+    int BH;        // query heads B * H
+    int H;         // query heads per batch entry
+    int group;     // query heads per K/V head (1 = multi-head, H = multi-query)
     int T;
     int causal;
     float c_log2;  // scale * log2(e)
@@ -171,7 +176,7 @@ __device__ __forceinline__ void exp_pairs(const float (&s)[128], float2 c2, floa
 }
 
 struct UnitInfo {
-    int bh, i0;
+    int bh, kvh, i0;  // query head, its K/V head, first query row
     int n[2];
     int niter;
 };
@@ -205,6 +210,7 @@ __device__ __forceinline__ int unit_of(const FusedParams &p, int k, UnitInfo &u)
         u.bh = pid / p.nqb;
         qb = pid - u.bh * p.nqb;
     }
+    u.kvh = (u.bh / p.H) * (p.H / p.group) + (u.bh % p.H) / p.group;
     u.i0 = qb * 256;
     const int r1 = u.i0 + 128;
     if (p.causal) {
@@ -340,12 +346,12 @@ __global__ void __launch_bounds__(384, 1)
                     qph[t] ^= 1u;
                 }
                 if (!ok) break;
-                ok = load_kv(&tmK, 0, u.bh);
+                ok = load_kv(&tmK, 0, u.kvh);
                 for (int j = 1; ok && j < u.niter; ++j) {
-                    ok = load_kv(&tmK, j, u.bh);
-                    if (ok) ok = load_kv(&tmV, j - 1, u.bh);
+                    ok = load_kv(&tmK, j, u.kvh);
+                    if (ok) ok = load_kv(&tmV, j - 1, u.kvh);
                 }
-                if (ok) ok = load_kv(&tmV, u.niter - 1, u.bh);
+                if (ok) ok = load_kv(&tmV, u.niter - 1, u.kvh);
             }
             if (!ok) {
                 *abort_flag = 1;

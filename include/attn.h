@@ -67,6 +67,19 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
              int d_h, int causal, float scale, void *stream);
 
 /*
+ * Fused forward with grouped-query attention: the H query heads of a batch
+ * entry share H_kv K/V heads, query head h reading K/V head h / (H / H_kv)
+ * ("FlashAttention -- avoid writing the giant intermediate", "Return to the
+ * incident": grouped-query attention changes how the head structure sizes the
+ * persistent K/V state).
+ *   q, o : bf16 [B, H, T, d_h];  k, v : bf16 [B, H_kv, T, d_h];  lse : fp32 [B, H, T]
+ *   H_kv >= 1 and H % H_kv == 0 (H_kv = H is attn_fwd, H_kv = 1 multi-query).
+ * Other arguments, errors and asynchrony as attn_fwd.
+ */
+int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                 int H_kv, int T, int d_h, int causal, float scale, void *stream);
+
+/*
  * Unfused attention forward: three kernels with the T x T intermediates in
  * device memory, as in the materialised path ("Storing and Rereading Large
  * Intermediate Matrices"):

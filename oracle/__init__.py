@@ -48,6 +48,11 @@ def _load():
         lib.oracle_head_scores_probs.restype = None
         lib.oracle_head_scores_probs.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_double, P, ctypes.c_int64, P, P, P]
+        lib.oracle_attn_fwd_gqa.restype = ctypes.c_int
+        lib.oracle_attn_fwd_gqa.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, P, ctypes.c_int64, P,
+                                            ctypes.c_int64, P, P, ctypes.c_int]
         lib.oracle_attn_fwd.restype = ctypes.c_int
         lib.oracle_attn_fwd.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_double, P, ctypes.c_int64, P,
@@ -117,4 +122,31 @@ def attn_fwd(q_bits, k_bits, v_bits, causal: bool, scale: float, heads=None, row
                                  int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError("oracle_attn_fwd: bad argument")
+    return o, lse
+
+
+def attn_fwd_gqa(q_bits, k_bits, v_bits, causal: bool, scale: float, heads=None, rows=None,
+                 nthreads: int | None = None):
+    """Grouped-query attention forward in float64.
+
+    q_bits: uint16 [B, H, T, D]; k_bits/v_bits: uint16 [B, H_kv, T, D] with
+    H % H_kv == 0; query head h reads K/V head h // (H // H_kv).  Returns
+    (o, lse) with o [nheads, nrows, D] and lse [nheads, nrows] over flat query
+    heads b*H + h."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    B, H, T, D = q.shape
+    H_kv = k.shape[1]
+    h = None if heads is None else np.ascontiguousarray(heads, dtype=np.int64)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nh = B * H if h is None else h.shape[0]
+    nr = T if r is None else r.shape[0]
+    o = np.empty((nh, nr, D), dtype=np.float64)
+    lse = np.empty((nh, nr), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), B, H, H_kv, T, D,
+                                     int(bool(causal)), float(scale), _ptr(h), nh, _ptr(r), nr,
+                                     _ptr(o), _ptr(lse), int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd_gqa: bad argument")
     return o, lse

@@ -101,6 +101,7 @@ void oracle_head_scores_probs(const uint16_t *q, const uint16_t *k, int T, int D
 
 typedef struct {
     const uint16_t *q, *k, *v;
+    int64_t H, group;  /* query heads per batch entry; query heads per K/V head */
     int T, D, causal;
     double scale;
     const int64_t *heads;
@@ -131,10 +132,14 @@ static void *worker(void *arg)
         if (nr > ORACLE_ROW_BLOCK) nr = ORACLE_ROW_BLOCK;
         for (int64_t r = 0; r < nr; ++r)
             blk_rows[r] = jb->rows ? jb->rows[r0 + r] : r0 + r;
+        /* grouped-query attention: query head h of batch entry b reads K/V
+         * head b * (H / group) + h / group (group = 1: every head its own) */
+        const int64_t kvh = (bh / jb->H) * (jb->H / jb->group) + (bh % jb->H) / jb->group;
         const size_t head_off = (size_t)bh * (size_t)T * (size_t)D;
-        oracle_head_scores_probs(jb->q + head_off, jb->k + head_off, T, D, jb->causal, jb->scale,
+        const size_t kv_off = (size_t)kvh * (size_t)T * (size_t)D;
+        oracle_head_scores_probs(jb->q + head_off, jb->k + kv_off, T, D, jb->causal, jb->scale,
                                  blk_rows, nr, S, P, L);
-        const uint16_t *vh = jb->v + head_off;
+        const uint16_t *vh = jb->v + kv_off;
         for (int64_t r = 0; r < nr; ++r) {
             size_t orow = ((size_t)hi * (size_t)jb->nrows + (size_t)(r0 + r));
             double *out = jb->o + orow * (size_t)D;
@@ -158,19 +163,22 @@ static void *worker(void *arg)
     return NULL;
 }
 
-/* Attention forward for a subset of heads and rows.
- *   q, k, v : bf16 bit patterns, [B*H, T, D] contiguous (head bh at bh*T*D).
- *   heads   : flat head indices bh in [0, B*H), or NULL for all heads (then
- *             nheads must be B*H).
- *   rows    : query rows in [0, T), or NULL for all rows (nrows must be T).
+/* Attention forward with grouped-query heads, for a subset of heads and rows.
+ *   q       : bf16 bit patterns [B, H, T, D] (query head bh = b*H + h at bh*T*D).
+ *   k, v    : bf16 bit patterns [B, H_kv, T, D]; query head h of batch entry b
+ *             reads K/V head b*H_kv + h / (H / H_kv).
+ *   heads   : flat query-head indices in [0, B*H), or NULL for all heads.
+ *   rows    : query rows in [0, T), or NULL for all rows.
  *   o       : double [nheads, nrows, D];  lse : double [nheads, nrows].
- *   nthreads: worker threads (>= 1).
  * Returns 0, or -1 on a bad argument. */
-int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t BH, int T,
-                    int D, int causal, double scale, const int64_t *heads, int64_t nheads,
-                    const int64_t *rows, int64_t nrows, double *o, double *lse, int nthreads)
+int oracle_attn_fwd_gqa(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                        int64_t H, int64_t H_kv, int T, int D, int causal, double scale,
+                        const int64_t *heads, int64_t nheads, const int64_t *rows, int64_t nrows,
+                        double *o, double *lse, int nthreads)
 {
-    if (!q || !k || !v || !o || !lse || BH < 1 || T < 1 || D < 1 || nheads < 1 || nrows < 1)
+    const int64_t BH = B * H;
+    if (!q || !k || !v || !o || !lse || B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || T < 1 ||
+        D < 1 || nheads < 1 || nrows < 1)
         return -1;
     if (!heads && nheads != BH) return -1;
     if (!rows && nrows != T) return -1;
@@ -185,8 +193,8 @@ int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int
     job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     for (int t = 0; t < nthreads; ++t) {
-        job_t j = {q, k, v, T, D, causal, scale, heads, nheads, rows, nrows, o, lse, nitems, iph, t,
-                   nthreads};
+        job_t j = {q, k, v, H, H / H_kv, T, D, causal, scale, heads, nheads, rows, nrows, o, lse,
+                   nitems, iph, t, nthreads};
         jobs[t] = j;
     }
     for (int t = 1; t < nthreads; ++t)
@@ -197,4 +205,14 @@ int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int
     free(jobs);
     free(th);
     return 0;
+}
+
+/* Attention forward (every head has its own K and V) for a subset of heads
+ * and rows: q, k, v are [B*H, T, D]; the grouped form with H = H_kv = BH. */
+int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t BH, int T,
+                    int D, int causal, double scale, const int64_t *heads, int64_t nheads,
+                    const int64_t *rows, int64_t nrows, double *o, double *lse, int nthreads)
+{
+    return oracle_attn_fwd_gqa(q, k, v, 1, BH, BH, T, D, causal, scale, heads, nheads, rows,
+                               nrows, o, lse, nthreads);
 }

@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import exact_attention_124_b200 as attn
-from attn_inputs import WORKLOADS, make_qkv, make_workload, sample_rows
+import oracle
+from attn_inputs import WORKLOADS, bf16_bits, make_qkv, make_workload, sample_rows
 from tests.gpu_util import check_full, gather, oracle_ref, require_gpu, run_fused, to_dev
 from tests.parity import assert_parity, compare
 
@@ -145,3 +146,26 @@ def test_every_exp_split_every_element(split, D):
             assert_parity(st, f"split={split} D={D} causal={causal}")
     finally:
         attn.set_exp_split(prev)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("B,H,H_kv,T,causal", [(2, 8, 2, 700, True), (1, 8, 1, 513, False),
+                                               (2, 4, 4, 384, True), (1, 16, 2, 1024, False)])
+def test_grouped_query_every_element(B, H, H_kv, T, causal, D):
+    q, _, _ = make_qkv(B, H, T, D, 9300 + H + T)
+    _, k, v = make_qkv(B, H_kv, T, D, 9400 + H_kv + T)
+    o, lse = attn.fwd_gqa(*to_dev(q, k, v), causal)
+    assert attn.last_error() == 0
+    ro, rl = oracle.attn_fwd_gqa(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal,
+                                 1 / math.sqrt(D))
+    st = compare(o.double().cpu().numpy().reshape(ro.shape),
+                 lse.double().cpu().numpy().reshape(rl.shape), ro, rl)
+    assert_parity(st, f"gqa B={B} H={H} H_kv={H_kv} T={T} D={D}")
+
+
+def test_gqa_with_one_group_per_head_is_attn_fwd():
+    q, k, v = to_dev(*make_qkv(2, 4, 640, 128, 77))
+    o1, l1 = attn.fwd(q, k, v, True)
+    o2, l2 = attn.fwd_gqa(q, k, v, True)
+    assert attn.last_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -163,3 +163,40 @@ def test_bad_arguments_raise():
         oracle.attn_fwd(q, k, v, True, 1.0, rows=[8])
     with pytest.raises(ValueError):
         oracle.attn_fwd(q, k, v, True, 1.0, heads=[1])
+
+
+def _brute_gqa(qf, kf, vf, causal, scale, group):
+    """Definition of grouped-query attention at 50 digits: query head h uses
+    K/V head h // group."""
+    H = qf.shape[0]
+    outs, lses = [], []
+    for h in range(H):
+        o, l = _brute(qf[h], kf[h // group], vf[h // group], causal, scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+@pytest.mark.parametrize("H,H_kv,causal", [(4, 2, True), (6, 1, False), (4, 4, True)])
+def test_gqa_brute_force_tiny(H, H_kv, causal):
+    T, D = 9, 4
+    q, _, _ = make_qkv(1, H, T, D, 300 + H)
+    _, k, v = make_qkv(1, H_kv, T, D, 400 + H_kv)
+    scale = 0.5
+    o, lse = oracle.attn_fwd_gqa(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
+    bo, bl = _brute_gqa(_f64(bf16_bits(q[0])), _f64(bf16_bits(k[0])), _f64(bf16_bits(v[0])),
+                        causal, scale, H // H_kv)
+    assert np.max(np.abs(o - bo)) < 1e-13 and np.max(np.abs(lse - bl)) < 1e-12
+
+
+def test_gqa_batch_entries_use_their_own_kv_heads():
+    # B = 2: batch entry 1's query heads must read batch entry 1's K/V heads
+    B, H, H_kv, T, D = 2, 4, 2, 33, 8
+    q, _, _ = make_qkv(B, H, T, D, 51)
+    _, k, v = make_qkv(B, H_kv, T, D, 52)
+    o, lse = oracle.attn_fwd_gqa(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 0.3)
+    for b in range(B):
+        for h in range(H):
+            ob, lb = oracle.attn_fwd(bf16_bits(q[b, h]), bf16_bits(k[b, h // 2]),
+                                     bf16_bits(v[b, h // 2]), True, 0.3)
+            assert np.array_equal(o[b * H + h], ob[0]) and np.array_equal(lse[b * H + h], lb[0])
