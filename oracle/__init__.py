@@ -53,6 +53,16 @@ def _load():
                                             ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_double, P, ctypes.c_int64, P,
                                             ctypes.c_int64, P, P, ctypes.c_int]
+        lib.oracle_head_fwd_f64.restype = None
+        lib.oracle_head_fwd_f64.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, P, P]
+        lib.oracle_head_bwd_f64.restype = None
+        lib.oracle_head_bwd_f64.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, P, P, P]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_double, P, P, P, ctypes.c_int]
         lib.oracle_attn_fwd.restype = ctypes.c_int
         lib.oracle_attn_fwd.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_double, P, ctypes.c_int64, P,
@@ -150,3 +160,49 @@ def attn_fwd_gqa(q_bits, k_bits, v_bits, causal: bool, scale: float, heads=None,
     if rc != 0:
         raise ValueError("oracle_attn_fwd_gqa: bad argument")
     return o, lse
+
+
+def head_fwd_f64(q, k, v, causal: bool, scale: float):
+    """Forward of one head on float64 inputs [T, D]; returns (o, lse)."""
+    q, k, v = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v))
+    T, D = q.shape
+    o = np.empty((T, D))
+    lse = np.empty(T)
+    _load().oracle_head_fwd_f64(_ptr(q), _ptr(k), _ptr(v), T, D, int(bool(causal)),
+                                float(scale), _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def head_bwd_f64(q, k, v, dout, causal: bool, scale: float):
+    """Gradients (dq, dk, dv) of one head on float64 inputs [T, D]."""
+    q, k, v, g = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v, dout))
+    T, D = q.shape
+    dq, dk, dv = (np.empty((T, D)) for _ in range(3))
+    _load().oracle_head_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g), T, D, int(bool(causal)),
+                                float(scale), _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
+def attn_bwd(q_bits, k_bits, v_bits, dout_bits, causal: bool, scale: float,
+             nthreads: int | None = None):
+    """Gradients in float64 from bf16 inputs.  q/dout [B, H, T, D], k/v
+    [B, H_kv, T, D].  Returns dq [B, H, T, D] and dk, dv [B, H_kv, T, D]
+    (summed over the query heads of each group)."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    g = np.ascontiguousarray(dout_bits, dtype=np.uint16)
+    B, H, T, D = q.shape
+    H_kv = k.shape[1]
+    dq = np.empty((B, H, T, D))
+    dkh = np.empty((B, H, T, D))
+    dvh = np.empty((B, H, T, D))
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, H, H_kv, T, D,
+                                 int(bool(causal)), float(scale), _ptr(dq), _ptr(dkh), _ptr(dvh),
+                                 int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd: bad argument")
+    grp = H // H_kv
+    dk = dkh.reshape(B, H_kv, grp, T, D).sum(axis=2)
+    dv = dvh.reshape(B, H_kv, grp, T, D).sum(axis=2)
+    return dq, dk, dv

@@ -216,3 +216,172 @@ int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int
     return oracle_attn_fwd_gqa(q, k, v, 1, BH, BH, T, D, causal, scale, heads, nheads, rows,
                                nrows, o, lse, nthreads);
 }
+
+/* ------------------------------------------------------------------------
+ * Backward pass (gradients of attention), float64, one head at a time.
+ *
+ * With P the row softmax of the masked, scaled scores and O = P V, the
+ * gradients of a loss with output gradient dO are (chain rule through the
+ * three steps of the definition):
+ *   dV = P^T dO
+ *   dP = dO V^T
+ *   dS = P o (dP - rowsum(P o dP))        (softmax Jacobian, o = elementwise;
+ *                                          masked entries have P = 0, so dS = 0)
+ *   dQ = scale * dS K,    dK = scale * dS^T Q
+ * This recomputes S and P from Q and K, the recomputation the pages name as
+ * the cost of not storing the intermediates ("Attention Mechanism:
+ * Computation & Memory Patterns", section 4).  S, P, dP and dS are
+ * materialised for the whole head.
+ * ------------------------------------------------------------------------ */
+
+/* Forward of one head on double inputs (q, k, v: [T, D] row-major); o [T, D],
+ * lse [T].  The same definition as the bf16 entry points. */
+void oracle_head_fwd_f64(const double *q, const double *k, const double *v, int T, int D,
+                         int causal, double scale, double *o, double *lse)
+{
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    double *p = (double *)malloc(sizeof(double) * (size_t)T);
+    unsigned char *mk = (unsigned char *)malloc((size_t)T);
+    for (int i = 0; i < T; ++i) {
+        for (int j = 0; j < T; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += q[(size_t)i * D + c] * k[(size_t)j * D + c];
+            s[j] = scale * acc;
+            mk[j] = (unsigned char)(causal && j > i);
+        }
+        lse[i] = oracle_softmax_row(s, mk, T, p);
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < T; ++j)
+                if (p[j] != 0.0) acc += p[j] * v[(size_t)j * D + c];
+            o[(size_t)i * D + c] = acc;
+        }
+    }
+    free(s);
+    free(p);
+    free(mk);
+}
+
+/* Gradients of one head on double inputs: dq, dk, dv [T, D]. */
+void oracle_head_bwd_f64(const double *q, const double *k, const double *v, const double *dout,
+                         int T, int D, int causal, double scale, double *dq, double *dk,
+                         double *dv)
+{
+    const size_t TT = (size_t)T * (size_t)T;
+    double *P = (double *)malloc(sizeof(double) * TT);
+    double *dP = (double *)malloc(sizeof(double) * TT);
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    unsigned char *mk = (unsigned char *)malloc((size_t)T);
+    for (int i = 0; i < T; ++i) { /* S and P, row by row */
+        for (int j = 0; j < T; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += q[(size_t)i * D + c] * k[(size_t)j * D + c];
+            s[j] = scale * acc;
+            mk[j] = (unsigned char)(causal && j > i);
+        }
+        oracle_softmax_row(s, mk, T, P + (size_t)i * T);
+    }
+    for (int i = 0; i < T; ++i) /* dP = dO V^T */
+        for (int j = 0; j < T; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += dout[(size_t)i * D + c] * v[(size_t)j * D + c];
+            dP[(size_t)i * T + j] = acc;
+        }
+    for (int i = 0; i < T; ++i) { /* dS = P o (dP - rowsum(P o dP)), stored over dP */
+        double r = 0.0;
+        for (int j = 0; j < T; ++j)
+            r += P[(size_t)i * T + j] * dP[(size_t)i * T + j];
+        for (int j = 0; j < T; ++j)
+            dP[(size_t)i * T + j] = P[(size_t)i * T + j] * (dP[(size_t)i * T + j] - r);
+    }
+    for (int j = 0; j < T; ++j) /* dV = P^T dO, dK = scale dS^T Q */
+        for (int c = 0; c < D; ++c) {
+            double av = 0.0, ak = 0.0;
+            for (int i = 0; i < T; ++i) {
+                av += P[(size_t)i * T + j] * dout[(size_t)i * D + c];
+                ak += dP[(size_t)i * T + j] * q[(size_t)i * D + c];
+            }
+            dv[(size_t)j * D + c] = av;
+            dk[(size_t)j * D + c] = scale * ak;
+        }
+    for (int i = 0; i < T; ++i) /* dQ = scale dS K */
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < T; ++j)
+                acc += dP[(size_t)i * T + j] * k[(size_t)j * D + c];
+            dq[(size_t)i * D + c] = scale * acc;
+        }
+    free(P);
+    free(dP);
+    free(s);
+    free(mk);
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    int64_t H, group, BH;
+    int T, D, causal;
+    double scale;
+    double *dq, *dk, *dv;
+    int tid, nthreads;
+} bwd_job_t;
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job_t *jb = (bwd_job_t *)arg;
+    const int T = jb->T, D = jb->D;
+    const size_t n = (size_t)T * (size_t)D;
+    double *q = (double *)malloc(sizeof(double) * n), *k = (double *)malloc(sizeof(double) * n);
+    double *v = (double *)malloc(sizeof(double) * n), *g = (double *)malloc(sizeof(double) * n);
+    double *dk = (double *)malloc(sizeof(double) * n), *dv = (double *)malloc(sizeof(double) * n);
+    for (int64_t bh = jb->tid; bh < jb->BH; bh += jb->nthreads) {
+        const int64_t kvh = (bh / jb->H) * (jb->H / jb->group) + (bh % jb->H) / jb->group;
+        for (size_t e = 0; e < n; ++e) {
+            q[e] = bf16_to_f64(jb->q[(size_t)bh * n + e]);
+            g[e] = bf16_to_f64(jb->dout[(size_t)bh * n + e]);
+            k[e] = bf16_to_f64(jb->k[(size_t)kvh * n + e]);
+            v[e] = bf16_to_f64(jb->v[(size_t)kvh * n + e]);
+        }
+        oracle_head_bwd_f64(q, k, v, g, T, D, jb->causal, jb->scale, jb->dq + (size_t)bh * n, dk,
+                            dv);
+        /* per query head: dk, dv of its K/V head; the caller sums over a group */
+        memcpy(jb->dk + (size_t)bh * n, dk, sizeof(double) * n);
+        memcpy(jb->dv + (size_t)bh * n, dv, sizeof(double) * n);
+    }
+    free(q); free(k); free(v); free(g); free(dk); free(dv);
+    return NULL;
+}
+
+/* Gradients for all heads.  q, dout: bf16 [B, H, T, D]; k, v: bf16
+ * [B, H_kv, T, D].  dq: double [B, H, T, D]; dk, dv: double [B, H, T, D] per
+ * QUERY head (the contribution of that head to its K/V head's gradient;
+ * summing over the heads of a group gives dK and dV of the K/V head).
+ * Returns 0, or -1 on a bad argument. */
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                    int64_t B, int64_t H, int64_t H_kv, int T, int D, int causal, double scale,
+                    double *dq, double *dk, double *dv, int nthreads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || B < 1 || H < 1 || H_kv < 1 ||
+        H % H_kv != 0 || T < 1 || D < 1)
+        return -1;
+    const int64_t BH = B * H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > BH) nthreads = (int)BH;
+    bwd_job_t *jobs = (bwd_job_t *)calloc((size_t)nthreads, sizeof(bwd_job_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        bwd_job_t j = {q, k, v, dout, H, H / H_kv, BH, T, D, causal, scale, dq, dk, dv, t, nthreads};
+        jobs[t] = j;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        pthread_create(&th[t], NULL, bwd_worker, &jobs[t]);
+    bwd_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(jobs);
+    free(th);
+    return 0;
+}
