@@ -58,8 +58,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["fused", "unfused"], default="fused",
-                    help="unfused: the three-kernel materialised path (S and P in HBM)")
+    ap.add_argument("--path", choices=["fused", "unfused", "backward"], default="fused",
+                    help="unfused: the three-kernel materialised path (S and P in HBM); "
+                         "backward: the gradient kernels (recomputing S and P)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's B")
     ap.add_argument("--exp-split", type=int, default=None,
                     help="fused kernel variant: column pairs of every 8 whose exponentials run "
@@ -285,6 +286,8 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     if args.path == "unfused":
         return run_unfused(args, w, world, rank, local, peaks, peak_src)
+    if args.path == "backward":
+        return run_backward(args, w, world, rank, local, peaks, peak_src)
 
     # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
     q, k, v = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)
@@ -449,6 +452,63 @@ def run_unfused(args, w, world, rank, local, peaks, peak_src):
                          "algorithmic_bytes": nbytes, "traffic": None},
             "clocks": sampler.summary(), "gpu_launches": 3 * args.steps,
             "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0 if status == 0 else 1
+
+
+def run_backward(args, w, world, rank, local, peaks, peak_src):
+    """Times attn_bwd (row statistics + dK/dV kernel + dQ kernel) per step.
+    Counted FLOPs: 10*T^2*d_h per head (five T x T x d_h products: S, dP, dV,
+    dK, dQ), halved when causal; the kernels actually run seven (S and dP are
+    recomputed once per gradient kernel), reported beside it."""
+    import torch
+    import exact_attention_124_b200 as attn
+    dev = torch.device("cuda", local)
+    if w.T % 128:
+        raise SystemExit("the backward pass needs T to be a multiple of 128")
+    q, k, v = [t.to(dev) for t in make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)]
+    g = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank) + 7)[0].to(dev)
+    o, lse = attn.fwd(q, k, v, w.causal, w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(w.B * w.H * w.T * 8, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.bwd(q, k, v, o, lse, g, w.causal, w.scale, dq=dq, dk=dk, dv=dv, ws=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if attn.last_error() != 0:
+        raise SystemExit("device error during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    status = attn.last_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    counted = 2.5 * counted_flops(w)
+    peak = float(peaks["bf16_tflops"])
+    if rank == 0:
+        value = whole_job_tflops(counted, world, ms)
+        line = {
+            "metric": "attention bwd TFLOP/s (10*T^2*d_h per head, halved causal)",
+            "path": "backward", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "shape": w.describe(), "seed": w.seed},
+            "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak,
+                         "unit": "TFLOP/s", "frac": value / world / peak,
+                         "peak_source": f"{peak_src} bf16_tflops",
+                         "executed_tflops": 1.4 * value / world},
+            "clocks": sampler.summary(), "gpu_launches": 3 * args.steps, "device_status": status,
         }
         print(json.dumps(line), flush=True)
     return 0 if status == 0 else 1

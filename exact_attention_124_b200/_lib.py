@@ -41,6 +41,9 @@ def load_library():
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_bwd_workspace_bytes.argtypes = [I, I, I]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_fwd_unfused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_unfused_workspace_bytes.argtypes = [I, I, I]
@@ -56,7 +59,7 @@ def load_library():
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
-    for name in ("attn_fwd", "attn_fwd_gqa", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
+    for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
                  "attn_selftest_last_wait_site", "attn_selftest_set_exp_split"):
@@ -137,6 +140,31 @@ def fwd_gqa(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None,
                           B, H, H_kv, T, D, int(bool(causal)), float(scale), _stream(stream))
     _check(rc, "attn_fwd_gqa")
     return o, lse
+
+
+def bwd(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, dq=None, dk=None,
+        dv=None, ws=None, stream=None):
+    """Backward pass: gradients (dq, dk, dv) from the forward's o and lse and
+    the output gradient dout.  q/o/dout [B, H, T, d_h], k/v [B, H_kv, T, d_h],
+    T a multiple of 128."""
+    lib = load_library()
+    B, H, T, D = _shape(q)
+    H_kv = int(k.shape[1])
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _want(t, n)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        ws = torch.empty(int(lib.attn_bwd_workspace_bytes(B, H, T)), dtype=torch.uint8,
+                         device=q.device)
+    rc = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                      B, H, H_kv, T, D, int(bool(causal)), float(scale), _stream(stream))
+    _check(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def unfused_workspace_bytes(B: int, H: int, T: int) -> int:

@@ -11,6 +11,7 @@
 
 #include "attn.h"
 #include "attn_selftest.h"
+#include "backward.cuh"
 #include "fused_fwd.cuh"
 #include "selftest.cuh"
 #include "unfused.cuh"
@@ -96,6 +97,10 @@ int device_ready(int *sms_out)
         if (major != 10 || minor != 0 || sms < 1) return ATTN_ERR_NO_DEVICE;
         if (get_encoder() != ATTN_OK) return ATTN_ERR_LAUNCH;
         bool ok = true;
+        ok &= set_smem(attn::bwd_dkdv_kernel<64>, attn::BwdCfg<64>::SMEM);
+        ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
+        ok &= set_smem(attn::bwd_dq_kernel<64>, attn::BwdCfg<64>::SMEM);
+        ok &= set_smem(attn::bwd_dq_kernel<128>, attn::BwdCfg<128>::SMEM);
         ok &= fused_all_ready<64>();
         ok &= fused_all_ready<128>();
         ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
@@ -228,9 +233,72 @@ int launch_unfused(const void *q, const void *k, const void *v, void *o, float *
     return launch_status();
 }
 
+template <int D>
+int launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+               const void *dout, void *dq, void *dk, void *dv, void *ws, int B, int H, int H_kv,
+               int T, int causal, float scale, cudaStream_t stream)
+{
+    using C = attn::BwdCfg<D>;
+    const int BH = B * H, BHkv = B * H_kv;
+    CUtensorMap mq, mk, mv, mg;
+    if (make_map(&mq, q, D, T, BH, 128) || make_map(&mg, dout, D, T, BH, 128) ||
+        make_map(&mk, k, D, T, BHkv, 128) || make_map(&mv, v, D, T, BHkv, 128))
+        return ATTN_ERR_LAUNCH;
+    auto *stats = static_cast<float2 *>(ws);
+    const long long rows = (long long)BH * T;
+    attn::bwd_stats_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse,
+        stats, rows);
+    if (launch_status()) return ATTN_ERR_LAUNCH;
+    attn::BwdParams p;
+    p.stats = stats;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.group = H / H_kv;
+    p.T = T;
+    p.nq = T / 128;
+    p.causal = causal;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.limit_ns = kWaitLimitNs;
+    p.out_a = static_cast<__nv_bfloat16 *>(dk);
+    p.out_b = static_cast<__nv_bfloat16 *>(dv);
+    attn::bwd_dkdv_kernel<D><<<dim3(T / 128, BHkv), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
+    if (launch_status()) return ATTN_ERR_LAUNCH;
+    p.out_a = static_cast<__nv_bfloat16 *>(dq);
+    p.out_b = nullptr;
+    attn::bwd_dq_kernel<D><<<dim3(T / 128, BH), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t attn_bwd_workspace_bytes(int B, int H, int T)
+{
+    if (B < 1 || H < 1 || T < 1) return 0;
+    return (size_t)B * H * T * 8;
+}
+
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dout, void *dq, void *dk, void *dv, void *ws, int B, int H, int H_kv,
+             int T, int d_h, int causal, float scale, void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, T, d_h, causal, scale);
+    if (rc) return rc;
+    if (!dout || !dq || !dk || !dv || !ws) return ATTN_ERR_NULL;
+    if (misaligned(dout) || misaligned(dq) || misaligned(dk) || misaligned(dv) || misaligned(ws))
+        return ATTN_ERR_ALIGN;
+    if (H_kv < 1 || H % H_kv != 0 || T % 128 != 0 || (long long)B * H > 65535)
+        return ATTN_ERR_BAD_SHAPE;
+    if ((rc = device_ready(nullptr))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64
+               ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, H_kv, T, causal, scale, s)
+               : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, H_kv, T, causal, scale, s);
+}
+
 
 int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
              int d_h, int causal, float scale, void *stream)

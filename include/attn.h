@@ -80,6 +80,28 @@ int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *ls
                  int H_kv, int T, int d_h, int causal, float scale, void *stream);
 
 /*
+ * Backward pass (gradients) of the fused forward, recomputing S and P from Q,
+ * K and the forward's lse instead of reading stored intermediates
+ * ("Attention Mechanism: Computation & Memory Patterns", section 4):
+ *   dV = P^T dO,  dS = P o (dP - D) with dP = dO V^T and D_i = sum_c dO_ic O_ic,
+ *   dQ = scale dS K,  dK = scale dS^T Q   (K/V heads sum over their group).
+ *   q, o, dout : in,  bf16 [B, H, T, d_h]   (o, lse: the forward's outputs)
+ *   k, v       : in,  bf16 [B, H_kv, T, d_h]
+ *   lse        : in,  fp32 [B, H, T]
+ *   dq         : out, bf16 [B, H, T, d_h];  dk, dv : out, bf16 [B, H_kv, T, d_h]
+ *   ws         : caller-owned device workspace of attn_bwd_workspace_bytes()
+ *                bytes (per-row statistics; contents on return unspecified)
+ * T must be a multiple of 128; H % H_kv == 0; B * H <= 65535.  Other
+ * arguments, errors and asynchrony as attn_fwd.
+ */
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dout, void *dq, void *dk, void *dv, void *ws, int B, int H, int H_kv,
+             int T, int d_h, int causal, float scale, void *stream);
+
+/* Bytes of attn_bwd's workspace: B * H * T * 8.  0 on bad sizes. */
+size_t attn_bwd_workspace_bytes(int B, int H, int T);
+
+/*
  * Unfused attention forward: three kernels with the T x T intermediates in
  * device memory, as in the materialised path ("Storing and Rereading Large
  * Intermediate Matrices"):
