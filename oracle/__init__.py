@@ -63,6 +63,10 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64,
                                         ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_double, P, P, P, ctypes.c_int]
+        lib.oracle_attn_decode.restype = ctypes.c_int
+        lib.oracle_attn_decode.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P]
         lib.oracle_attn_fwd.restype = ctypes.c_int
         lib.oracle_attn_fwd.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_double, P, ctypes.c_int64, P,
@@ -206,3 +210,21 @@ def attn_bwd(q_bits, k_bits, v_bits, dout_bits, causal: bool, scale: float,
     dk = dkh.reshape(B, H_kv, grp, T, D).sum(axis=2)
     dv = dvh.reshape(B, H_kv, grp, T, D).sum(axis=2)
     return dq, dk, dv
+
+
+def attn_decode(q_bits, k_bits, v_bits, causal: bool, scale: float):
+    """Decode attention in float64: q [B, H, Tq, D] against a cache k/v
+    [B, H_kv, Tk, D]; query i sits at position Tk - Tq + i.  Returns
+    (o [B, H, Tq, D], lse [B, H, Tq])."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    B, H, Tq, D = q.shape
+    H_kv, Tk = k.shape[1], k.shape[2]
+    o = np.empty((B, H, Tq, D))
+    lse = np.empty((B, H, Tq))
+    rc = _load().oracle_attn_decode(_ptr(q), _ptr(k), _ptr(v), B, H, H_kv, Tq, Tk, D,
+                                    int(bool(causal)), float(scale), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_decode: bad argument")
+    return o, lse

@@ -385,3 +385,52 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
     free(th);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Decode: Tq new queries against Tk cached keys/values (Tq <= Tk).  Query i
+ * sits at position Tk - Tq + i; with the causal mask it sees keys
+ * j <= Tk - Tq + i (itself and earlier tokens), otherwise all Tk keys.
+ * Grouped-query heads as in oracle_attn_fwd_gqa.  Same definition as the
+ * forward (S and P of each query row materialised over all Tk keys).
+ *   q : bf16 [B, H, Tq, D];  k, v : bf16 [B, H_kv, Tk, D]
+ *   o : double [B, H, Tq, D];  lse : double [B, H, Tq]
+ * ------------------------------------------------------------------------ */
+int oracle_attn_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                       int64_t H, int64_t H_kv, int Tq, int Tk, int D, int causal, double scale,
+                       double *o, double *lse)
+{
+    if (!q || !k || !v || !o || !lse || B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Tq < 1 ||
+        Tk < Tq || D < 1)
+        return -1;
+    const int64_t group = H / H_kv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)Tk);
+    double *p = (double *)malloc(sizeof(double) * (size_t)Tk);
+    unsigned char *mk = (unsigned char *)malloc((size_t)Tk);
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t kvh = (bh / H) * H_kv + (bh % H) / group;
+        const uint16_t *qh = q + (size_t)bh * Tq * D;
+        const uint16_t *kh = k + (size_t)kvh * Tk * D;
+        const uint16_t *vh = v + (size_t)kvh * Tk * D;
+        for (int i = 0; i < Tq; ++i) {
+            const int pos = Tk - Tq + i;
+            for (int j = 0; j < Tk; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < D; ++c)
+                    acc += bf16_to_f64(qh[(size_t)i * D + c]) * bf16_to_f64(kh[(size_t)j * D + c]);
+                s[j] = scale * acc;
+                mk[j] = (unsigned char)(causal && j > pos);
+            }
+            lse[(size_t)bh * Tq + i] = oracle_softmax_row(s, mk, Tk, p);
+            for (int c = 0; c < D; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < Tk; ++j)
+                    if (p[j] != 0.0) acc += p[j] * bf16_to_f64(vh[(size_t)j * D + c]);
+                o[((size_t)bh * Tq + i) * D + c] = acc;
+            }
+        }
+    }
+    free(s);
+    free(p);
+    free(mk);
+    return 0;
+}

@@ -200,3 +200,43 @@ def test_gqa_batch_entries_use_their_own_kv_heads():
             ob, lb = oracle.attn_fwd(bf16_bits(q[b, h]), bf16_bits(k[b, h // 2]),
                                      bf16_bits(v[b, h // 2]), True, 0.3)
             assert np.array_equal(o[b * H + h], ob[0]) and np.array_equal(lse[b * H + h], lb[0])
+
+
+def test_decode_with_tq_equal_tk_is_the_forward():
+    B, H, H_kv, T, D = 1, 4, 2, 40, 8
+    q, _, _ = make_qkv(B, H, T, D, 81)
+    _, k, v = make_qkv(B, H_kv, T, D, 82)
+    for causal in (True, False):
+        o, l = oracle.attn_decode(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 0.4)
+        of, lf = oracle.attn_fwd_gqa(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 0.4)
+        assert np.array_equal(o.reshape(of.shape), of) and np.array_equal(l.reshape(lf.shape), lf)
+
+
+def test_decode_last_rows_of_causal_forward():
+    # Tq new tokens at the end of a Tk-token sequence: the same rows as the
+    # last Tq rows of the causal forward over all Tk tokens
+    B, H, Tk, Tq, D = 1, 2, 37, 5, 8
+    q, k, v = make_qkv(B, H, Tk, D, 83)
+    o, l = oracle.attn_decode(bf16_bits(q[:, :, Tk - Tq:]), bf16_bits(k), bf16_bits(v), True, 0.3)
+    of, lf = oracle.attn_fwd(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 0.3)
+    assert np.array_equal(o.reshape(B * H, Tq, D), of[:, Tk - Tq:])
+    assert np.array_equal(l.reshape(B * H, Tq), lf[:, Tk - Tq:])
+
+
+def test_decode_brute_force_tiny():
+    B, H, H_kv, Tq, Tk, D = 1, 2, 1, 3, 11, 4
+    q, _, _ = make_qkv(B, H, Tq, D, 84)
+    _, k, v = make_qkv(B, H_kv, Tk, D, 85)
+    o, l = oracle.attn_decode(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 0.5)
+    mpmath.mp.dps = 50
+    qf, kf, vf = _f64(bf16_bits(q[0])), _f64(bf16_bits(k[0, 0])), _f64(bf16_bits(v[0, 0]))
+    for h in range(H):
+        for i in range(Tq):
+            js = range(Tk - Tq + i + 1)
+            e = [mpmath.exp(mpmath.mpf(0.5) * mpmath.fsum(mpmath.mpf(qf[h, i, c]) * mpmath.mpf(kf[j, c])
+                                                          for c in range(D))) for j in js]
+            den = mpmath.fsum(e)
+            for c in range(D):
+                ref = float(mpmath.fsum(e[n] * mpmath.mpf(vf[j, c]) for n, j in enumerate(js)) / den)
+                assert abs(o[0, h, i, c] - ref) < 1e-13
+            assert abs(l[0, h, i] - float(mpmath.log(den))) < 1e-13
