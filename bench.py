@@ -58,9 +58,13 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["fused", "unfused", "backward"], default="fused",
+    ap.add_argument("--decode-tq", type=int, default=1, help="decode: new queries per head")
+    ap.add_argument("--decode-hkv", type=int, default=0,
+                    help="decode: K/V heads (0: the workload's H / 4)")
+    ap.add_argument("--path", choices=["fused", "unfused", "backward", "decode"], default="fused",
                     help="unfused: the three-kernel materialised path (S and P in HBM); "
-                         "backward: the gradient kernels (recomputing S and P)")
+                         "backward: the gradient kernels (recomputing S and P); "
+                         "decode: --decode-tq queries against a cache of the workload's T tokens")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's B")
     ap.add_argument("--exp-split", type=int, default=None,
                     help="fused kernel variant: column pairs of every 8 whose exponentials run "
@@ -288,6 +292,8 @@ def run_ours(args):
         return run_unfused(args, w, world, rank, local, peaks, peak_src)
     if args.path == "backward":
         return run_backward(args, w, world, rank, local, peaks, peak_src)
+    if args.path == "decode":
+        return run_decode(args, w, world, rank, local, peaks, peak_src)
 
     # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
     q, k, v = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)
@@ -509,6 +515,69 @@ def run_backward(args, w, world, rank, local, peaks, peak_src):
                          "peak_source": f"{peak_src} bf16_tflops",
                          "executed_tflops": 1.4 * value / world},
             "clocks": sampler.summary(), "gpu_launches": 3 * args.steps, "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0 if status == 0 else 1
+
+
+def run_decode(args, w, world, rank, local, peaks, peak_src):
+    """Times attn_fwd_decode (split-KV partials + merge): --decode-tq queries
+    per head against a K/V cache of the workload's T tokens with H_kv heads.
+    HBM-bound: algorithmic bytes = the K/V cache read once + Q read + O, lse
+    written."""
+    import torch
+    import exact_attention_124_b200 as attn
+    dev = torch.device("cuda", local)
+    H_kv = args.decode_hkv or max(1, w.H // 4)
+    Tq, Tk = args.decode_tq, w.T
+    q = make_qkv(w.B, w.H, Tq, w.D, rank_seed(w, rank))[0].to(dev)
+    _, k, v = make_qkv(w.B, H_kv, Tk, w.D, rank_seed(w, rank) + 1)
+    k, v = k.to(dev), v.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, Tq), dtype=torch.float32, device=dev)
+    lib = attn.load_library()
+    ws = torch.empty(int(lib.attn_decode_workspace_bytes(w.B, w.H, H_kv, Tq, Tk, w.D, 0)),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.fwd_decode(q, k, v, True, w.scale, splits=0, o=o, lse=lse, ws=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if attn.last_error() != 0:
+        raise SystemExit("device error during warm-up")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2, between steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize()
+    sampler.start()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    status = attn.last_error()
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world, dev)
+    nbytes = 2 * k.numel() * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    if rank == 0:
+        line = {
+            "metric": "attention decode: effective HBM GB/s (K/V cache read once)",
+            "path": "decode", "value": gbs * world, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"decode B={w.B} H={w.H} H_kv={H_kv} Tq={Tq} Tk={Tk} "
+                                   f"d_h={w.D} causal", "l2": "256 MB flush before each step"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic_bytes": nbytes},
+            "clocks": sampler.summary(), "gpu_launches": 2 * args.steps, "device_status": status,
         }
         print(json.dumps(line), flush=True)
     return 0 if status == 0 else 1

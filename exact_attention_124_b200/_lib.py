@@ -42,6 +42,9 @@ def load_library():
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
     lib.attn_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_fwd_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd_workspace_bytes.argtypes = [I, I, I]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_fwd_unfused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P]
@@ -59,7 +62,7 @@ def load_library():
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
-    for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
+    for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_decode", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
                  "attn_selftest_last_wait_site", "attn_selftest_set_exp_split"):
@@ -165,6 +168,32 @@ def bwd(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, dq=None
                       B, H, H_kv, T, D, int(bool(causal)), float(scale), _stream(stream))
     _check(rc, "attn_bwd")
     return dq, dk, dv
+
+
+def fwd_decode(q, k, v, causal: bool, scale: float | None = None, splits: int = 0, o=None,
+               lse=None, ws=None, stream=None):
+    """Decode forward: q [B, H, Tq, d_h] against a cache k/v [B, H_kv, Tk, d_h]
+    (query i at position Tk - Tq + i), split-KV over ``splits`` key ranges
+    (0: automatic).  Returns (o, lse)."""
+    lib = load_library()
+    B, H, Tq, D = _shape(q)
+    _, H_kv, Tk, _ = _shape(k)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t, n)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        nbytes = int(lib.attn_decode_workspace_bytes(B, H, H_kv, Tq, Tk, D, int(splits)))
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    rc = lib.attn_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), ws.data_ptr(), B, H, H_kv, Tq, Tk, D,
+                             int(bool(causal)), float(scale), int(splits), _stream(stream))
+    _check(rc, "attn_fwd_decode")
+    return o, lse
 
 
 def unfused_workspace_bytes(B: int, H: int, T: int) -> int:

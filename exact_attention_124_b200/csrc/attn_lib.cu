@@ -12,6 +12,7 @@
 #include "attn.h"
 #include "attn_selftest.h"
 #include "backward.cuh"
+#include "decode.cuh"
 #include "fused_fwd.cuh"
 #include "selftest.cuh"
 #include "unfused.cuh"
@@ -101,6 +102,8 @@ int device_ready(int *sms_out)
         ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<64>, attn::BwdCfg<64>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<128>, attn::BwdCfg<128>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<64>, attn::DecCfg<64>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<128>, attn::DecCfg<128>::SMEM);
         ok &= fused_all_ready<64>();
         ok &= fused_all_ready<128>();
         ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
@@ -271,9 +274,94 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     return launch_status();
 }
 
+// Split-KV geometry of the decode path: key tiles of 128, tiles per split,
+// number of splits (every split gets at least one tile).  splits <= 0 picks
+// enough splits for about two CTAs per SM.
+void decode_geometry(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms, int &nkt,
+                     int &chunk, int &eff)
+{
+    nkt = (Tk + 127) / 128;
+    const int rows = (H / H_kv) * Tq;
+    const long long ctas = (long long)B * H_kv * ((rows + 127) / 128);
+    if (splits <= 0) splits = (int)((2LL * sms + ctas - 1) / ctas);
+    if (splits > nkt) splits = nkt;
+    if (splits < 1) splits = 1;
+    chunk = (nkt + splits - 1) / splits;
+    eff = (nkt + chunk - 1) / chunk;
+}
+
+template <int D>
+int launch_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
+                  int B, int H, int H_kv, int Tq, int Tk, int causal, float scale, int splits,
+                  cudaStream_t stream, int sms)
+{
+    using C = attn::DecCfg<D>;
+    int nkt, chunk, eff;
+    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, nkt, chunk, eff);
+    const long long nrows = (long long)B * H * Tq;
+    CUtensorMap mq, mk, mv;
+    if (make_map(&mq, q, D, (uint64_t)nrows, 1, 128) ||
+        make_map(&mk, k, D, Tk, (uint64_t)B * H_kv, 128) ||
+        make_map(&mv, v, D, Tk, (uint64_t)B * H_kv, 128))
+        return ATTN_ERR_LAUNCH;
+    attn::DecodeParams p;
+    p.part_o = static_cast<float *>(ws);
+    p.part_lse = p.part_o + (size_t)eff * nrows * D;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.group = H / H_kv;
+    p.Tq = Tq;
+    p.Tk = Tk;
+    p.causal = causal;
+    p.rows = p.group * Tq;
+    p.nkt = nkt;
+    p.chunk = chunk;
+    p.splits = eff;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.limit_ns = kWaitLimitNs;
+    const dim3 grid(eff, B * H_kv, (p.rows + 127) / 128);
+    attn::decode_partial_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    if (launch_status()) return ATTN_ERR_LAUNCH;
+    attn::decode_combine_kernel<D><<<(unsigned)((nrows + 7) / 8), 256, 0, stream>>>(
+        p.part_o, p.part_lse, static_cast<__nv_bfloat16 *>(o), lse, nrows, eff);
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int d_h, int splits)
+{
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Tq < 1 || Tk < Tq ||
+        (d_h != 64 && d_h != 128))
+        return 0;
+    int sms = 0;
+    if (splits <= 0 && device_ready(&sms)) return 0;
+    int nkt, chunk, eff;
+    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, nkt, chunk, eff);
+    return (size_t)eff * B * H * Tq * (size_t)(d_h + 1) * 4;
+}
+
+int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
+                    int B, int H, int H_kv, int Tq, int Tk, int d_h, int causal, float scale,
+                    int splits, void *stream)
+{
+    int rc = validate(q, k, v, o, lse, B, H, Tq, d_h, causal, scale);
+    if (rc) return rc;
+    if (!ws) return ATTN_ERR_NULL;
+    if (misaligned(ws)) return ATTN_ERR_ALIGN;
+    if (H_kv < 1 || H % H_kv != 0 || Tk < Tq || (long long)B * H_kv > 65535 ||
+        (long long)B * H * Tq > INT_MAX || (long long)B * H_kv * Tk > INT_MAX)
+        return ATTN_ERR_BAD_SHAPE;
+    int sms = 0;
+    if ((rc = device_ready(&sms))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d_h == 64
+               ? launch_decode<64>(q, k, v, o, lse, ws, B, H, H_kv, Tq, Tk, causal, scale, splits, s, sms)
+               : launch_decode<128>(q, k, v, o, lse, ws, B, H, H_kv, Tq, Tk, causal, scale, splits, s, sms);
+}
+
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T)
 {

@@ -80,6 +80,29 @@ int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *ls
                  int H_kv, int T, int d_h, int causal, float scale, void *stream);
 
 /*
+ * Decode forward: Tq new queries against a K/V cache of Tk >= Tq tokens,
+ * query i at position Tk - Tq + i (causal: it sees keys 0 .. Tk - Tq + i;
+ * "FlashAttention -- avoid writing the giant intermediate": persistent K/V
+ * state in cached decoding, measured apart from prefill).  Grouped-query heads
+ * as attn_fwd_gqa.  The key range is split across CTAs (split-KV) and the
+ * splits' partial results are merged by their log-sum-exp.
+ *   q, o   : bf16 [B, H, Tq, d_h];  k, v : bf16 [B, H_kv, Tk, d_h]
+ *   lse    : out, fp32 [B, H, Tq]
+ *   ws     : caller-owned device workspace of attn_decode_workspace_bytes()
+ *            bytes for the same sizes and splits (partial outputs)
+ *   splits : key splits (clamped to [1, ceil(Tk / 128)]); <= 0 picks enough
+ *            for about two CTAs per SM
+ * Other arguments, errors and asynchrony as attn_fwd.
+ */
+int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
+                    int B, int H, int H_kv, int Tq, int Tk, int d_h, int causal, float scale,
+                    int splits, void *stream);
+
+/* Bytes of attn_fwd_decode's workspace for these sizes and splits; 0 on bad
+ * sizes (or, with splits <= 0, without a device). */
+size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int d_h, int splits);
+
+/*
  * Backward pass (gradients) of the fused forward, recomputing S and P from Q,
  * K and the forward's lse instead of reading stored intermediates
  * ("Attention Mechanism: Computation & Memory Patterns", section 4):

@@ -1,0 +1,62 @@
+"""Parity of the split-KV decode path (attn_fwd_decode) with the float64
+oracle: Tq new queries against a Tk-token K/V cache, query i at position
+Tk - Tq + i ("FlashAttention -- avoid writing the giant intermediate": the
+persistent K/V state of cached decoding).  Same bounds as the prefill path."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_124_b200 as attn
+import oracle
+from attn_inputs import bf16_bits, make_qkv
+from tests.gpu_util import require_gpu, to_dev
+from tests.parity import assert_parity, compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _case(B, H, H_kv, Tq, Tk, D, causal, splits, seed):
+    q, _, _ = make_qkv(B, H, Tq, D, seed)
+    _, k, v = make_qkv(B, H_kv, Tk, D, seed + 1)
+    o, lse = attn.fwd_decode(*to_dev(q, k, v), causal, splits=splits)
+    assert attn.last_error() == 0
+    ro, rl = oracle.attn_decode(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 1 / math.sqrt(D))
+    return compare(o.double().cpu().numpy(), lse.double().cpu().numpy(), ro, rl)
+
+
+@pytest.mark.parametrize("B,H,H_kv,Tq,Tk,D,causal,splits", [
+    (2, 8, 2, 1, 4096, 128, True, 0),
+    (2, 8, 2, 1, 4096, 128, True, 1),
+    (2, 8, 2, 1, 4096, 128, True, 7),
+    (1, 4, 4, 16, 1000, 64, True, 3),
+    (1, 4, 4, 16, 1000, 64, False, 0),
+    (1, 32, 8, 64, 2048, 128, True, 4),
+    (3, 6, 3, 5, 333, 128, True, 2),
+    (1, 2, 1, 1, 1, 64, True, 0),
+])
+def test_decode_every_element(B, H, H_kv, Tq, Tk, D, causal, splits):
+    st = _case(B, H, H_kv, Tq, Tk, D, causal, splits, 7700 + Tq + Tk + D + splits)
+    assert_parity(st, f"decode B={B} H={H} H_kv={H_kv} Tq={Tq} Tk={Tk} D={D} splits={splits}")
+
+
+def test_decode_with_tq_equal_tk_matches_prefill():
+    q, k, v = to_dev(*make_qkv(1, 4, 512, 128, 91))
+    o1, l1 = attn.fwd(q, k, v, True)
+    o2, l2 = attn.fwd_decode(q, k, v, True, splits=2)
+    assert attn.last_error() == 0
+    assert (o1.double() - o2.double()).abs().max().item() < 2e-2
+    assert (l1 - l2).abs().max().item() < 1e-3
+
+
+def test_decode_rejects_cache_shorter_than_queries():
+    q = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 4, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(attn.AttnError):
+        attn.fwd_decode(q, k, k, True, ws=torch.empty(64, dtype=torch.uint8, device="cuda"))
