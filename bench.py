@@ -51,7 +51,7 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -208,35 +208,42 @@ def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> f
 
 # ---------------------------------------------------------------------------- CPU oracle
 def oracle_sample(w, seconds: float, seed_offset: int = 0):
-    """Time the float64 oracle on an evenly spread row sample of head 0 of
-    workload ``w`` sized to about ``seconds`` of CPU work.  Returns
-    (TFLOP/s in the metric's counting, seconds, rows, threads, description)."""
+    """Time the float64 oracle on a sample of workload ``w`` sized to about
+    ``seconds`` of CPU work: evenly spaced query rows of one head, and whole
+    heads once one head is not enough.  Returns (TFLOP/s in the metric's
+    counting, seconds, rows, threads, description)."""
     import numpy as np
     import oracle
-    q, k, v = make_qkv(1, 1, w.T, w.D, w.seed + seed_offset, w.qk_mult)
-    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
     threads = oracle.default_threads()
+    max_heads = min(w.heads, 64)
+    q, k, v = make_qkv(1, max_heads, w.T, w.D, w.seed + seed_offset, w.qk_mult)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
 
-    def run(nrows):
+    def run(nheads, nrows):
         step = max(1, w.T // nrows)
         rows = np.arange(step // 2, w.T, step, dtype=np.int64)[:nrows]
         t0 = time.perf_counter()
-        oracle.attn_fwd(qb, kb, vb, w.causal, w.scale, rows=rows, nthreads=threads)
+        oracle.attn_fwd(qb, kb, vb, w.causal, w.scale, heads=np.arange(nheads), rows=rows,
+                        nthreads=threads)
         dt = time.perf_counter() - t0
         # the metric's counting: 4*d per visible key (QK^T and PV), per row
         vis = (rows + 1) if w.causal else np.full(rows.shape, w.T)
-        return rows, dt, float(4.0 * w.D * vis.sum())
+        return rows, dt, float(4.0 * w.D * vis.sum()) * nheads
 
-    n = max(threads, 32)
-    for _ in range(3):  # calibrate the sample size to the time budget
-        rows, dt, fl = run(n)
-        if dt >= 0.6 * seconds or n >= w.T:
+    nheads, n = 1, max(threads, 32)
+    for _ in range(5):  # calibrate the sample size to the time budget
+        rows, dt, fl = run(nheads, n)
+        if dt >= 0.6 * seconds or (n >= w.T and nheads >= max_heads):
             break
-        n = int(min(w.T, max(n + 1, n * seconds / max(dt, 1e-6))))
-    desc = (f"{len(rows)} evenly spaced query rows of one head (T={w.T}, d_h={w.D}, "
+        grow = seconds / max(dt, 1e-6)
+        if n < w.T:
+            n = int(min(w.T, max(n + 1, n * grow)))
+        else:
+            nheads = int(min(max_heads, max(nheads + 1, nheads * grow)))
+    desc = (f"{len(rows)} evenly spaced query rows of {nheads} head(s) (T={w.T}, d_h={w.D}, "
             f"{'causal' if w.causal else 'full'}), float64, {threads} threads; FLOPs counted "
             f"as 4*d_h per visible key")
-    return fl / dt / 1e12, dt, len(rows), threads, desc
+    return fl / dt / 1e12, dt, len(rows) * nheads, threads, desc
 
 
 def run_reference(args):
