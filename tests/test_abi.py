@@ -100,3 +100,37 @@ def test_mma_order_switch(lib):
     assert attn.set_mma_order(prev) == 1
     with pytest.raises(ValueError):
         attn.set_mma_order(3)
+
+
+def test_gqa_rejects_bad_head_grouping(lib):
+    # H = 6 query heads cannot share H_kv = 4 K/V heads
+    assert lib.attn_fwd_gqa(A, A, A, A, A, 1, 6, 4, 128, 64, 1, 0.125, None) == 3
+    assert lib.attn_fwd_gqa(A, A, A, A, A, 1, 6, 0, 128, 64, 1, 0.125, None) == 3
+    assert lib.attn_fwd_gqa(None, A, A, A, A, 1, 6, 3, 128, 64, 1, 0.125, None) == 1
+
+
+def test_backward_rejects_bad_arguments(lib):
+    ok = [A, A, A, A, A, A, A, A, A, A, 1, 4, 2, 256, 128, 1, 0.125, None]
+    bad = list(ok); bad[9] = None            # no workspace
+    assert lib.attn_bwd(*bad) == 1
+    bad = list(ok); bad[13] = 200            # T not a multiple of 128
+    assert lib.attn_bwd(*bad) == 3
+    bad = list(ok); bad[12] = 3              # 4 heads over 3 K/V heads
+    assert lib.attn_bwd(*bad) == 3
+    bad = list(ok); bad[6] = A + 8           # misaligned dq
+    assert lib.attn_bwd(*bad) == 4
+    bad = list(ok); bad[14] = 80             # unsupported head size
+    assert lib.attn_bwd(*bad) == 2
+    assert attn.load_library().attn_bwd_workspace_bytes(2, 4, 256) == 2 * 4 * 256 * 8
+
+
+def test_decode_rejects_bad_arguments(lib):
+    ok = [A, A, A, A, A, A, 1, 8, 2, 4, 1024, 128, 1, 0.125, 0, None]
+    bad = list(ok); bad[5] = None            # no workspace
+    assert lib.attn_fwd_decode(*bad) == 1
+    bad = list(ok); bad[10] = 2              # cache shorter than the new queries
+    assert lib.attn_fwd_decode(*bad) == 3
+    bad = list(ok); bad[8] = 3               # 8 heads over 3 K/V heads
+    assert lib.attn_fwd_decode(*bad) == 3
+    # workspace size with explicit splits needs no device: 4 splits x rows x (d + 1) floats
+    assert lib.attn_decode_workspace_bytes(1, 8, 2, 4, 1024, 128, 4) == 4 * 1 * 8 * 4 * 129 * 4
