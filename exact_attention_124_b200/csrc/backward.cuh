@@ -48,7 +48,7 @@ struct BwdCfg {
     static constexpr int OFF_FIX = 0;           // the stationary pair of tiles
     static constexpr int OFF_RING = 2 * TILE;
     static constexpr int OFF_BAR = OFF_RING + NST * STAGE;
-    static constexpr int NBAR = 1 + 2 * NST + 3 + 1;
+    static constexpr int NBAR = 1 + 2 * NST + 4 + 1;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
     static constexpr int THREADS = 256;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -110,8 +110,8 @@ struct BwdSmem {
         b_full = bar + 8;                 // [NST]
         b_empty = b_full + 8 * C::NST;    // [NST]
         b_sfull = b_empty + 8 * C::NST;
-        b_pfull = b_sfull + 8;
-        b_done = b_pfull + 8;
+        b_pfull = b_sfull + 8;            // [2]: columns 0-63 / 64-127 written
+        b_done = b_pfull + 16;
         b_drain = b_done + 8;
         tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
         abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -130,6 +130,7 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D> &sm, int warp)
         }
         mbar_init(sm.b_sfull, 1);
         mbar_init(sm.b_pfull, 128);
+        mbar_init(sm.b_pfull + 8, 128);
         mbar_init(sm.b_done, 1);
         mbar_init(sm.b_drain, 1);
         *sm.abort_flag = 0;
@@ -152,12 +153,14 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D> &sm, int warp)
 // S columns in the dQ kernel).  Chunk c writes columns [16c, 16c + 16), all of
 // which earlier chunks (or this one) have already read.  PER_COLUMN: rows are
 // keys and the statistics come per query column from shared memory; else rows
-// are queries and the row's own statistics are st_row.
+// are queries and the row's own statistics are st_row.  Each half of the
+// columns is signalled on its own barrier (b_half, b_half + 8) as soon as it
+// is in TMEM, so the MMAs that consume it can start.
 template <bool PER_COLUMN, bool WRITE_P>
 __device__ __forceinline__ void bwd_elementwise(uint32_t tS, uint32_t tDP, float cl2,
                                                 const float2 *st_col, float2 st_row,
                                                 bool need_mask, int row_idx, int col0,
-                                                uint32_t tDS)
+                                                uint32_t tDS, uint32_t b_half)
 {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -189,6 +192,11 @@ __device__ __forceinline__ void bwd_elementwise(uint32_t tS, uint32_t tDP, float
         }
         if (WRITE_P) tmem_st16(tS + 16 * c, pk);
         tmem_st16(tDS + 16 * c, dk);
+        if (c & 1) {  // columns [0, 64) after chunk 1, [64, 128) after chunk 3
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(b_half + 8 * (c >> 1));
+        }
     }
 }
 
@@ -295,17 +303,23 @@ __global__ void __launch_bounds__(256, 1)
                            sw128_desc_join(gl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(sm.b_sfull);
-                if (!(ok = mbar_wait(sm.b_pfull, (uint32_t)n & 1u, lim, W_B_PFULL, sm.abort_flag))) break;
-                tc_fence_after_sync();
                 const uint32_t qm = sw128_desc_lo(st, C::SUB), gm = sw128_desc_lo(st + C::TILE, C::SUB);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO, dK += dS^T Q (16 queries each)
-                    const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
-                           sw128_desc_join(gm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
-                    mma_ts(tmem + C::TM_ACC1, tmem + C::TM_DP + 8 * kk,
-                           sw128_desc_join(qm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
+                for (int hh = 0; hh < 2; ++hh) {  // each half of the queries as soon as it is ready
+                    if (!(ok = mbar_wait(sm.b_pfull + 8 * hh, (uint32_t)n & 1u, lim, W_B_PFULL,
+                                         sm.abort_flag)))
+                        break;
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk) {  // dV += P^T dO, dK += dS^T Q
+                        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+                        mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
+                               sw128_desc_join(gm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
+                        mma_ts(tmem + C::TM_ACC1, tmem + C::TM_DP + 8 * kk,
+                               sw128_desc_join(qm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
+                    }
                 }
+                if (!ok) break;
                 tc_commit(sm.b_empty + 8 * s);
             }
             if (!ok) *sm.abort_flag = 1;
@@ -329,10 +343,7 @@ __global__ void __launch_bounds__(256, 1)
             const bool need_mask = p.causal && i == j;
             bwd_elementwise<true, true>(tmem + lane_off + C::TM_S, tmem + lane_off + C::TM_DP,
                                         p.c_log2, stc, make_float2(0.f, 0.f), need_mask, key,
-                                        128 * i, tmem + lane_off + C::TM_DP);
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(sm.b_pfull);
+                                        128 * i, tmem + lane_off + C::TM_DP, sm.b_pfull);
         }
         const bool w = ok && mbar_wait(sm.b_done, 0, lim, W_B_DONE, sm.abort_flag);
         if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
@@ -432,14 +443,20 @@ __global__ void __launch_bounds__(256, 1)
                            sw128_desc_join(vl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(sm.b_sfull);
-                if (!(ok = mbar_wait(sm.b_pfull, (uint32_t)jj & 1u, lim, W_B_PFULL, sm.abort_flag))) break;
-                tc_fence_after_sync();
                 const uint32_t km = sw128_desc_lo(st, C::SUB);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // dQ += dS K (16 keys each)
-                    mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
-                           sw128_desc_join(km + kk * (2048 >> 4), 1024), C::IDESC_ACC,
-                           (jj > 0 || kk > 0) ? 1u : 0u);
+                for (int hh = 0; hh < 2; ++hh) {  // each half of the keys as soon as it is ready
+                    if (!(ok = mbar_wait(sm.b_pfull + 8 * hh, (uint32_t)jj & 1u, lim, W_B_PFULL,
+                                         sm.abort_flag)))
+                        break;
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk)  // dQ += dS K (16 keys each)
+                        mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
+                               sw128_desc_join(km + kk * (2048 >> 4), 1024), C::IDESC_ACC,
+                               (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (!ok) break;
                 tc_commit(sm.b_empty + 8 * s);
             }
             if (!ok) *sm.abort_flag = 1;
@@ -458,10 +475,7 @@ __global__ void __launch_bounds__(256, 1)
             const bool need_mask = p.causal && jj == i;
             bwd_elementwise<false, false>(tmem + lane_off + C::TM_S, tmem + lane_off + C::TM_DP,
                                           p.c_log2, nullptr, st_row, need_mask, row, 128 * jj,
-                                          tmem + lane_off + C::TM_S);
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(sm.b_pfull);
+                                          tmem + lane_off + C::TM_S, sm.b_pfull);
         }
         const bool w = ok && mbar_wait(sm.b_done, 0, lim, W_B_DONE, sm.abort_flag);
         if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
