@@ -16,9 +16,16 @@
 //   bwd_dq_kernel     one CTA per (query head, 128 queries): loops over the key
 //                     blocks it sees; S and dP into TMEM, dS back as bf16,
 //                     dQ += dS K in TMEM
-// Warps: 0-3 elementwise (thread = TMEM lane = the stationary block's row),
-// warp 4 issues MMAs, warp 5 issues TMA copies, warps 6-7 idle.
-// TMEM: S/P [0,128), dP/dS [128,256), accumulators from 256.
+// Each 128-wide block of the moving operand is taken as two 64-wide halves,
+// half h in TMEM buffer h and handled by elementwise warpgroup h, so the
+// tensor cores compute one half's S/dP and accumulate the other's gradient
+// while a warpgroup does the elementwise step (a two-buffer ping-pong; TMEM
+// has room for two 64-column S/dP pairs next to the 2 d_h accumulator
+// columns, not for two 128-column ones).
+// Warps: 0-3 / 4-7 elementwise warpgroups 0 / 1 (thread = TMEM lane = the
+// stationary block's row), warp 8 issues MMAs, warp 9 issues TMA copies.
+// TMEM: buffer h = S/P [128h, 128h + 64), dP/dS [128h + 64, 128h + 128);
+// accumulators from 256.
 #pragma once
 
 #include "sm100.cuh"
@@ -48,12 +55,16 @@ struct BwdCfg {
     static constexpr int OFF_FIX = 0;           // the stationary pair of tiles
     static constexpr int OFF_RING = 2 * TILE;
     static constexpr int OFF_BAR = OFF_RING + NST * STAGE;
-    static constexpr int NBAR = 1 + 2 * NST + 4 + 1;
+    static constexpr int NBAR = 1 + 2 * NST + 4 + 2;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
-    static constexpr int THREADS = 256;
+    static constexpr int THREADS = 320;
+    static constexpr int MMA_WARP = 8, TMA_WARP = 9;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC0 = 256, TM_ACC1 = 256 + D;
-    static constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false);  // N = 128 rows of B
+    static constexpr uint32_t TM_ACC0 = 256, TM_ACC1 = 256 + D;
+    static constexpr int HALF = 64 * 128;       // 64 rows x 128 bytes of a SW128 block
+    __host__ __device__ static constexpr uint32_t tm_s(int h) { return 128u * h; }
+    __host__ __device__ static constexpr uint32_t tm_dp(int h) { return 128u * h + 64u; }
+    static constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 64, false);   // N = 64 rows of B
     static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);    // B MN-major, N = d_h
 };
 
@@ -109,8 +120,8 @@ struct BwdSmem {
         b_fix = bar;
         b_full = bar + 8;                 // [NST]
         b_empty = b_full + 8 * C::NST;    // [NST]
-        b_sfull = b_empty + 8 * C::NST;
-        b_pfull = b_sfull + 8;            // [2]: columns 0-63 / 64-127 written
+        b_sfull = b_empty + 8 * C::NST;   // [2]: S/dP of buffer h computed
+        b_pfull = b_sfull + 16;           // [2]: P/dS of buffer h written
         b_done = b_pfull + 16;
         b_drain = b_done + 8;
         tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
@@ -128,15 +139,16 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D> &sm, int warp)
             mbar_init(sm.b_full + 8 * s, 1);
             mbar_init(sm.b_empty + 8 * s, 1);
         }
-        mbar_init(sm.b_sfull, 1);
-        mbar_init(sm.b_pfull, 128);
-        mbar_init(sm.b_pfull + 8, 128);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(sm.b_sfull + 8 * h, 1);
+            mbar_init(sm.b_pfull + 8 * h, 128);
+        }
         mbar_init(sm.b_done, 1);
         mbar_init(sm.b_drain, 1);
         *sm.abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 4) {
+    if (warp == C::MMA_WARP) {
         tmem_alloc(smem_addr(sm.tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -146,24 +158,23 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D> &sm, int warp)
     return *sm.tmem_slot;
 }
 
-// Elementwise step of both kernels on one 128 x 128 block, one row per
+// Elementwise step of both kernels on one 128 x 64 half block, one row per
 // thread, 32 columns at a time: p = 2^(s c - lse2) (0 where masked) and
-// ds = p (dp - D).  With WRITE_P, P (bf16 pairs) goes over the first 64 S
-// columns; dS goes to tDS (over the dP columns in the dK/dV kernel, over the
-// S columns in the dQ kernel).  Chunk c writes columns [16c, 16c + 16), all of
-// which earlier chunks (or this one) have already read.  PER_COLUMN: rows are
-// keys and the statistics come per query column from shared memory; else rows
-// are queries and the row's own statistics are st_row.  Each half of the
-// columns is signalled on its own barrier (b_half, b_half + 8) as soon as it
-// is in TMEM, so the MMAs that consume it can start.
+// ds = p (dp - D).  With WRITE_P, P (bf16 pairs) goes over the first 32 S
+// columns of the buffer; dS goes to tDS (over the dP columns in the dK/dV
+// kernel, over the S columns in the dQ kernel).  Chunk c writes columns
+// [16c, 16c + 16), all of which this or the earlier chunk has already read.
+// PER_COLUMN: rows are keys and the statistics come per query column from
+// shared memory; else rows are queries and the row's own statistics are
+// st_row.  The buffer is signalled on b_pfull once all of it is in TMEM.
 template <bool PER_COLUMN, bool WRITE_P>
 __device__ __forceinline__ void bwd_elementwise(uint32_t tS, uint32_t tDP, float cl2,
                                                 const float2 *st_col, float2 st_row,
                                                 bool need_mask, int row_idx, int col0,
-                                                uint32_t tDS, uint32_t b_half)
+                                                uint32_t tDS, uint32_t b_pfull)
 {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tS + 32 * c, rs);
         tmem_ld32(tDP + 32 * c, rd);
@@ -192,20 +203,19 @@ __device__ __forceinline__ void bwd_elementwise(uint32_t tS, uint32_t tDP, float
         }
         if (WRITE_P) tmem_st16(tS + 16 * c, pk);
         tmem_st16(tDS + 16 * c, dk);
-        if (c & 1) {  // columns [0, 64) after chunk 1, [64, 128) after chunk 3
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(b_half + 8 * (c >> 1));
-        }
     }
+    tmem_wait_st();
+    tc_fence_before_sync();
+    mbar_arrive(b_pfull);
 }
 
-// Epilogue: rows of a TMEM accumulator (D fp32 columns) times `mul`, as bf16.
-template <int D>
+// Epilogue: 32-column chunks [C0, C1) of the rows of a TMEM accumulator times
+// `mul`, as bf16.
+template <int C0, int C1>
 __device__ __forceinline__ void store_rows(uint32_t tacc, float mul, __nv_bfloat16 *dst)
 {
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = C0; c < C1; ++c) {
         uint32_t r[32];
         tmem_ld32(tacc + 32 * c, r);
         tmem_wait_ld_regs(r);
@@ -220,11 +230,50 @@ __device__ __forceinline__ void store_rows(uint32_t tacc, float mul, __nv_bfloat
     }
 }
 
+// MMA issue order of both kernels, iteration n of the moving operand, halves
+// 0 and 1 in buffers 0 and 1:
+//   sdp(0,0) sdp(0,1) | acc(n,0) sdp(n+1,0) acc(n,1) [stage free] sdp(n+1,1) | ...
+// where sdp(n,h) computes S/dP of half h into buffer h (signalled on
+// b_sfull[h]) and acc(n,h) waits for warpgroup h's P/dS (b_pfull[h]) and
+// accumulates from it.  The tensor pipe runs in issue order, so sdp(n+1,h)
+// overwrites buffer h only after acc(n,h) has read it.  Each of the four
+// barriers completes once per iteration and its waiter has passed the
+// previous completion before the next can start, so parity n & 1 is exact.
+template <typename Sdp, typename Acc, typename Full>
+__device__ __forceinline__ bool bwd_mma_loop(int niter, uint32_t b_pfull, uint32_t b_empty,
+                                             uint64_t lim, volatile int *abort_flag, Sdp sdp,
+                                             Acc acc, Full wait_full, int nst)
+{
+    if (niter <= 0) return true;
+    if (!wait_full(0)) return false;
+    tc_fence_after_sync();
+    sdp(0, 0);
+    sdp(0, 1);
+    for (int n = 0; n < niter; ++n) {
+        const uint32_t par = (uint32_t)n & 1u;
+        if (!mbar_wait(b_pfull, par, lim, W_B_PFULL, abort_flag)) return false;
+        tc_fence_after_sync();
+        acc(n, 0);
+        const bool more = n + 1 < niter;
+        if (more) {
+            if (!wait_full(n + 1)) return false;
+            tc_fence_after_sync();
+            sdp(n + 1, 0);
+        }
+        if (!mbar_wait(b_pfull + 8, par, lim, W_B_PFULL, abort_flag)) return false;
+        tc_fence_after_sync();
+        acc(n, 1);
+        tc_commit(b_empty + 8 * (n % nst));
+        if (more) sdp(n + 1, 1);
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- dK, dV
 // grid: (T / 128 key blocks, B * H_kv); key block j = blockIdx.x (causal:
 // the lowest keys see the most queries, so the longest CTAs start first).
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const BwdParams p)
@@ -244,7 +293,7 @@ __global__ void __launch_bounds__(256, 1)
     const int niter = p.group * per_head;
     const uint32_t sK = sm.fix, sV = sm.fix + C::TILE;
 
-    if (warp == 5) {
+    if (warp == C::TMA_WARP) {
         if (lane == 0) {  // TMA: K_j, V_j once; then Q_i, dO_i, stats per iteration
             const uint64_t pol = policy_evict_last();
             mbar_arrive_expect_tx(sm.b_fix, 2 * C::TILE);
@@ -282,94 +331,96 @@ __global__ void __launch_bounds__(256, 1)
                     if ((armed >> s) & 1u) mbar_wait(sm.b_full + 8 * s, (armed_par >> s) & 1u, lim, W_B_STFULL);
             }
         }
-    } else if (warp == 4) {
+    } else if (warp == C::MMA_WARP) {
         if (lane == 0) {  // MMA issuer
             bool ok = mbar_wait(sm.b_fix, 0, lim, W_B_KV, sm.abort_flag);
             tc_fence_after_sync();
             const uint32_t kl = sw128_desc_lo(sK, 16), vl = sw128_desc_lo(sV, 16);
-            for (int n = 0; ok && n < niter; ++n) {
-                const int s = n % C::NST;
-                const uint32_t par = (uint32_t)(n / C::NST) & 1u;
-                if (!(ok = mbar_wait(sm.b_full + 8 * s, par, lim, W_B_STFULL, sm.abort_flag))) break;
-                tc_fence_after_sync();
-                const uint32_t st = sm.ring + s * C::STAGE;
+            auto wait_full = [&](int n) {
+                return mbar_wait(sm.b_full + 8 * (n % C::NST), (uint32_t)(n / C::NST) & 1u, lim,
+                                 W_B_STFULL, sm.abort_flag);
+            };
+            auto sdp = [&](int n, int h) {  // S^T = K Q_h^T, dP^T = V dO_h^T (64 queries)
+                const uint32_t st = sm.ring + (n % C::NST) * C::STAGE + h * C::HALF;
                 const uint32_t ql = sw128_desc_lo(st, 16), gl = sw128_desc_lo(st + C::TILE, 16);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T, dP^T = V dO^T
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4;
-                    mma_ss(tmem + C::TM_S, sw128_desc_join(kl + off, 1024),
+                    mma_ss(tmem + C::tm_s(h), sw128_desc_join(kl + off, 1024),
                            sw128_desc_join(ql + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
-                    mma_ss(tmem + C::TM_DP, sw128_desc_join(vl + off, 1024),
+                    mma_ss(tmem + C::tm_dp(h), sw128_desc_join(vl + off, 1024),
                            sw128_desc_join(gl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(sm.b_sfull);
+                tc_commit(sm.b_sfull + 8 * h);
+            };
+            auto acc = [&](int n, int h) {  // dV += P_h^T dO_h, dK += dS_h^T Q_h (16 queries each)
+                const uint32_t st = sm.ring + (n % C::NST) * C::STAGE;
                 const uint32_t qm = sw128_desc_lo(st, C::SUB), gm = sw128_desc_lo(st + C::TILE, C::SUB);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {  // each half of the queries as soon as it is ready
-                    if (!(ok = mbar_wait(sm.b_pfull + 8 * hh, (uint32_t)n & 1u, lim, W_B_PFULL,
-                                         sm.abort_flag)))
-                        break;
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk) {  // dV += P^T dO, dK += dS^T Q
-                        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-                        mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
-                               sw128_desc_join(gm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
-                        mma_ts(tmem + C::TM_ACC1, tmem + C::TM_DP + 8 * kk,
-                               sw128_desc_join(qm + kk * (2048 >> 4), 1024), C::IDESC_ACC, acc);
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t a = (n > 0 || h > 0 || kk > 0) ? 1u : 0u;
+                    const uint32_t boff = (uint32_t)(4 * h + kk) * (2048 >> 4);
+                    mma_ts(tmem + C::TM_ACC0, tmem + C::tm_s(h) + 8 * kk,
+                           sw128_desc_join(gm + boff, 1024), C::IDESC_ACC, a);
+                    mma_ts(tmem + C::TM_ACC1, tmem + C::tm_dp(h) + 8 * kk,
+                           sw128_desc_join(qm + boff, 1024), C::IDESC_ACC, a);
                 }
-                if (!ok) break;
-                tc_commit(sm.b_empty + 8 * s);
-            }
+            };
+            ok = ok && bwd_mma_loop(niter, sm.b_pfull, sm.b_empty, lim, sm.abort_flag, sdp, acc,
+                                    wait_full, C::NST);
             if (!ok) *sm.abort_flag = 1;
             tc_commit(sm.b_done);  // fires when every MMA issued above has completed
         }
-    } else if (warp < 4) {  // elementwise: thread = key row
-        const int kr = warp * 32 + lane;
+    } else if (warp < 8) {  // elementwise warpgroup h: thread = key row, queries of half h
+        const int h = warp >> 2;
+        const int kr = (warp & 3) * 32 + lane;
         const int key = 128 * j + kr;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
         for (int n = 0; ok && n < niter; ++n) {
             const int s = n % C::NST;
             const uint32_t par = (uint32_t)(n / C::NST) & 1u;
             const int i = i0 + n % per_head;
             bool w = mbar_wait(sm.b_full + 8 * s, par, lim, W_B_STFULL, sm.abort_flag);
-            w = w && mbar_wait(sm.b_sfull, (uint32_t)n & 1u, lim, W_B_SFULL, sm.abort_flag);
+            w = w && mbar_wait(sm.b_sfull + 8 * h, (uint32_t)n & 1u, lim, W_B_SFULL, sm.abort_flag);
             if (!(ok = __all_sync(0xffffffffu, w))) break;
             tc_fence_after_sync();
-            const float2 *stc =
-                reinterpret_cast<const float2 *>(sm.gbase + C::OFF_RING + s * C::STAGE + 2 * C::TILE);
+            const float2 *stc = reinterpret_cast<const float2 *>(sm.gbase + C::OFF_RING +
+                                                                 s * C::STAGE + 2 * C::TILE) +
+                                64 * h;
             const bool need_mask = p.causal && i == j;
-            bwd_elementwise<true, true>(tmem + lane_off + C::TM_S, tmem + lane_off + C::TM_DP,
+            bwd_elementwise<true, true>(tmem + lane_off + C::tm_s(h), tmem + lane_off + C::tm_dp(h),
                                         p.c_log2, stc, make_float2(0.f, 0.f), need_mask, key,
-                                        128 * i, tmem + lane_off + C::TM_DP, sm.b_pfull);
+                                        128 * i + 64 * h, tmem + lane_off + C::tm_dp(h),
+                                        sm.b_pfull + 8 * h);
         }
         const bool w = ok && mbar_wait(sm.b_done, 0, lim, W_B_DONE, sm.abort_flag);
         if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
             tc_fence_after_sync();
             const size_t orow = ((size_t)kvbh * p.T + key) * D;
-            store_rows<D>(tmem + lane_off + C::TM_ACC1, p.scale, p.out_a + orow);  // dK
-            store_rows<D>(tmem + lane_off + C::TM_ACC0, 1.f, p.out_b + orow);      // dV
+            if (h == 0)
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC1, p.scale, p.out_a + orow);  // dK
+            else
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC0, 1.f, p.out_b + orow);  // dV
         } else {
             *sm.abort_flag = 1;
         }
     }
-    if (warp == 4 && lane == 0 && *sm.abort_flag) {
+    if (warp == C::MMA_WARP && lane == 0 && *sm.abort_flag) {
         tc_commit(sm.b_drain);
         mbar_wait(sm.b_drain, 0, lim, W_B_DRAIN);
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 4) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- dQ
 // grid: (T / 128 query blocks, B * H); causal: the highest query block sees
 // the most keys and starts first.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const BwdParams p)
@@ -388,7 +439,7 @@ __global__ void __launch_bounds__(256, 1)
     const int nkb = p.causal ? i + 1 : p.nq;
     const uint32_t sQ = sm.fix, sG = sm.fix + C::TILE;
 
-    if (warp == 5) {
+    if (warp == C::TMA_WARP) {
         if (lane == 0) {  // TMA: Q_i, dO_i once; then K_j, V_j per iteration
             const uint64_t pol = policy_evict_last();
             mbar_arrive_expect_tx(sm.b_fix, 2 * C::TILE);
@@ -422,77 +473,78 @@ __global__ void __launch_bounds__(256, 1)
                     if ((armed >> s) & 1u) mbar_wait(sm.b_full + 8 * s, (armed_par >> s) & 1u, lim, W_B_STFULL);
             }
         }
-    } else if (warp == 4) {
+    } else if (warp == C::MMA_WARP) {
         if (lane == 0) {  // MMA issuer
             bool ok = mbar_wait(sm.b_fix, 0, lim, W_B_KV, sm.abort_flag);
             tc_fence_after_sync();
             const uint32_t ql = sw128_desc_lo(sQ, 16), gl = sw128_desc_lo(sG, 16);
-            for (int jj = 0; ok && jj < nkb; ++jj) {
-                const int s = jj % C::NST;
-                const uint32_t par = (uint32_t)(jj / C::NST) & 1u;
-                if (!(ok = mbar_wait(sm.b_full + 8 * s, par, lim, W_B_STFULL, sm.abort_flag))) break;
-                tc_fence_after_sync();
-                const uint32_t st = sm.ring + s * C::STAGE;
+            auto wait_full = [&](int jj) {
+                return mbar_wait(sm.b_full + 8 * (jj % C::NST), (uint32_t)(jj / C::NST) & 1u, lim,
+                                 W_B_STFULL, sm.abort_flag);
+            };
+            auto sdp = [&](int jj, int h) {  // S = Q K_h^T, dP = dO V_h^T (64 keys)
+                const uint32_t st = sm.ring + (jj % C::NST) * C::STAGE + h * C::HALF;
                 const uint32_t kl = sw128_desc_lo(st, 16), vl = sw128_desc_lo(st + C::TILE, 16);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {  // S = Q K^T, dP = dO V^T
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4;
-                    mma_ss(tmem + C::TM_S, sw128_desc_join(ql + off, 1024),
+                    mma_ss(tmem + C::tm_s(h), sw128_desc_join(ql + off, 1024),
                            sw128_desc_join(kl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
-                    mma_ss(tmem + C::TM_DP, sw128_desc_join(gl + off, 1024),
+                    mma_ss(tmem + C::tm_dp(h), sw128_desc_join(gl + off, 1024),
                            sw128_desc_join(vl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(sm.b_sfull);
-                const uint32_t km = sw128_desc_lo(st, C::SUB);
+                tc_commit(sm.b_sfull + 8 * h);
+            };
+            auto acc = [&](int jj, int h) {  // dQ += dS_h K_h (16 keys each)
+                const uint32_t km = sw128_desc_lo(sm.ring + (jj % C::NST) * C::STAGE, C::SUB);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {  // each half of the keys as soon as it is ready
-                    if (!(ok = mbar_wait(sm.b_pfull + 8 * hh, (uint32_t)jj & 1u, lim, W_B_PFULL,
-                                         sm.abort_flag)))
-                        break;
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk)  // dQ += dS K (16 keys each)
-                        mma_ts(tmem + C::TM_ACC0, tmem + C::TM_S + 8 * kk,
-                               sw128_desc_join(km + kk * (2048 >> 4), 1024), C::IDESC_ACC,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                if (!ok) break;
-                tc_commit(sm.b_empty + 8 * s);
-            }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + C::TM_ACC0, tmem + C::tm_s(h) + 8 * kk,
+                           sw128_desc_join(km + (uint32_t)(4 * h + kk) * (2048 >> 4), 1024),
+                           C::IDESC_ACC, (jj > 0 || h > 0 || kk > 0) ? 1u : 0u);
+            };
+            ok = ok && bwd_mma_loop(nkb, sm.b_pfull, sm.b_empty, lim, sm.abort_flag, sdp, acc,
+                                    wait_full, C::NST);
             if (!ok) *sm.abort_flag = 1;
             tc_commit(sm.b_done);
         }
-    } else if (warp < 4) {  // elementwise: thread = query row
-        const int qr = warp * 32 + lane;
+    } else if (warp < 8) {  // elementwise warpgroup h: thread = query row, keys of half h
+        const int h = warp >> 2;
+        const int qr = (warp & 3) * 32 + lane;
         const int row = 128 * i + qr;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float2 st_row = p.stats[(size_t)bh * p.T + row];
         bool ok = true;
         for (int jj = 0; ok && jj < nkb; ++jj) {
-            const bool w = mbar_wait(sm.b_sfull, (uint32_t)jj & 1u, lim, W_B_SFULL, sm.abort_flag);
+            const bool w = mbar_wait(sm.b_sfull + 8 * h, (uint32_t)jj & 1u, lim, W_B_SFULL, sm.abort_flag);
             if (!(ok = __all_sync(0xffffffffu, w))) break;
             tc_fence_after_sync();
             const bool need_mask = p.causal && jj == i;
-            bwd_elementwise<false, false>(tmem + lane_off + C::TM_S, tmem + lane_off + C::TM_DP,
-                                          p.c_log2, nullptr, st_row, need_mask, row, 128 * jj,
-                                          tmem + lane_off + C::TM_S, sm.b_pfull);
+            bwd_elementwise<false, false>(tmem + lane_off + C::tm_s(h), tmem + lane_off + C::tm_dp(h),
+                                          p.c_log2, nullptr, st_row, need_mask, row,
+                                          128 * jj + 64 * h, tmem + lane_off + C::tm_s(h),
+                                          sm.b_pfull + 8 * h);
         }
         const bool w = ok && mbar_wait(sm.b_done, 0, lim, W_B_DONE, sm.abort_flag);
         if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
             tc_fence_after_sync();
-            store_rows<D>(tmem + lane_off + C::TM_ACC0, p.scale, p.out_a + ((size_t)bh * p.T + row) * D);
+            __nv_bfloat16 *dst = p.out_a + ((size_t)bh * p.T + row) * D;
+            if (h == 0)  // the two warpgroups store the two halves of the d_h columns
+                store_rows<0, D / 64>(tmem + lane_off + C::TM_ACC0, p.scale, dst);
+            else
+                store_rows<D / 64, D / 32>(tmem + lane_off + C::TM_ACC0, p.scale, dst);
         } else {
             *sm.abort_flag = 1;
         }
     }
-    if (warp == 4 && lane == 0 && *sm.abort_flag) {
+    if (warp == C::MMA_WARP && lane == 0 && *sm.abort_flag) {
         tc_commit(sm.b_drain);
         mbar_wait(sm.b_drain, 0, lim, W_B_DRAIN);
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 4) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace attn
