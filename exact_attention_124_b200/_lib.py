@@ -62,10 +62,12 @@ def load_library():
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
+    lib.attn_selftest_decode_plan.argtypes = [I, I, I, I, I, I, I, P, I, P, I, P]
     for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_decode", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
-                 "attn_selftest_last_wait_site", "attn_selftest_set_exp_split"):
+                 "attn_selftest_last_wait_site", "attn_selftest_set_exp_split",
+                 "attn_selftest_decode_plan"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -173,7 +175,8 @@ def bwd(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, dq=None
 def fwd_decode(q, k, v, causal: bool, scale: float | None = None, splits: int = 0, o=None,
                lse=None, ws=None, stream=None):
     """Decode forward: q [B, H, Tq, d_h] against a cache k/v [B, H_kv, Tk, d_h]
-    (query i at position Tk - Tq + i), split-KV over ``splits`` key ranges
+    (query i at position Tk - Tq + i), split-KV over ``splits`` key ranges per head
+    (< 0: balanced ranges of all heads' tiles over the SMs)
     (0: automatic).  Returns (o, lse)."""
     lib = load_library()
     B, H, Tq, D = _shape(q)
@@ -261,6 +264,27 @@ def set_exp_split(pairs_of_8: int) -> int:
     if prev == -2:
         raise ValueError("exp split must be -1, 0, 2, 3 or 4")
     return prev
+
+
+def decode_plan(B: int, H: int, H_kv: int, Tq: int, Tk: int, splits: int, sms: int):
+    """Host-side work plan of attn_fwd_decode on a device with ``sms`` SMs
+    (no device needed): (segments, nseg, slots) with segments a list of
+    (cta_x, cta_y, cta_z, kvbh, row_block, first_tile, tiles, slot) tuples and
+    nseg[w] the partial slots the merge reads for head w."""
+    lib = load_library()
+    nrb = ((H // H_kv) * Tq + 127) // 128 if H_kv > 0 and H % H_kv == 0 else 0
+    heads = B * H_kv * nrb
+    slots = ctypes.c_int(0)
+    n = lib.attn_selftest_decode_plan(B, H, H_kv, Tq, Tk, splits, sms, None, 0, None, 0,
+                                      ctypes.byref(slots))
+    if n < 0:
+        raise ValueError("bad decode sizes")
+    segs = (ctypes.c_int * (8 * max(n, 1)))()
+    nseg = (ctypes.c_int * max(heads, 1))()
+    n2 = lib.attn_selftest_decode_plan(B, H, H_kv, Tq, Tk, splits, sms, segs, n, nseg, heads,
+                                       ctypes.byref(slots))
+    assert n2 == n
+    return ([tuple(segs[8 * i:8 * i + 8]) for i in range(n)], list(nseg[:heads]), slots.value)
 
 
 def fused_grid_ctas(B: int, H: int, T: int, D: int, causal: bool) -> int:

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -277,17 +278,71 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 // Split-KV geometry of the decode path: key tiles of 128, tiles per split,
 // number of splits (every split gets at least one tile).  splits <= 0 picks
 // enough splits for about two CTAs per SM.
-void decode_geometry(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms, int &nkt,
-                     int &chunk, int &eff)
+struct DecGeom {
+    int nkt, nrb, balanced, chunk, eff, G, slots;
+    long long tot;
+};
+
+// splits > 0: every head cut into `splits` key ranges (clamped to the tile
+// count), one CTA each.  splits < 0: balanced ranges of the (head, key tile)
+// list, one CTA per SM.  splits == 0: the fixed split that fills one wave of
+// CTAs (one per SM) if that keeps at least 85 % of the SMs busy -- no range
+// boundary inside a CTA, no second wave -- else balanced.
+void decode_geometry(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms, DecGeom &g)
 {
-    nkt = (Tk + 127) / 128;
-    const int rows = (H / H_kv) * Tq;
-    const long long ctas = (long long)B * H_kv * ((rows + 127) / 128);
-    if (splits <= 0) splits = (int)((2LL * sms + ctas - 1) / ctas);
-    if (splits > nkt) splits = nkt;
-    if (splits < 1) splits = 1;
-    chunk = (nkt + splits - 1) / splits;
-    eff = (nkt + chunk - 1) / chunk;
+    g.nkt = (Tk + 127) / 128;
+    g.nrb = ((H / H_kv) * Tq + 127) / 128;
+    g.tot = (long long)B * H_kv * g.nrb * g.nkt;
+    const long long heads = (long long)B * H_kv * g.nrb;
+    if (splits == 0) {
+        const long long s = std::min<long long>(sms / heads, g.nkt);
+        const long long chunk = s > 0 ? (g.nkt + s - 1) / s : 0;
+        const long long busy = s > 0 ? heads * ((g.nkt + chunk - 1) / chunk) : 0;
+        splits = (s > 0 && 100 * busy >= 85LL * sms) ? (int)s : -1;
+    }
+    if (splits < 0) {
+        g.balanced = 1;
+        g.G = (int)std::min<long long>(sms, g.tot);
+        const long long per = g.tot / g.G;  // tiles per CTA, rounded down (>= 1)
+        // a head's nkt consecutive tiles meet at most (nkt - 1) / per + 2 ranges
+        g.slots = (int)std::min<long long>(g.G, (g.nkt - 1) / per + 2);
+        g.chunk = 0;
+        g.eff = 0;
+    } else {
+        g.balanced = 0;
+        g.G = 0;
+        if (splits > g.nkt) splits = g.nkt;
+        g.chunk = (g.nkt + splits - 1) / splits;
+        g.eff = (g.nkt + g.chunk - 1) / g.chunk;
+        g.slots = g.eff;
+    }
+}
+
+// Kernel parameters of a decode launch (workspace pointers left null).
+attn::DecodeParams decode_params(int B, int H, int H_kv, int Tq, int Tk, int causal, float scale,
+                                 const DecGeom &g)
+{
+    attn::DecodeParams p;
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
+    p.nrows = (long long)B * H * Tq;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.group = H / H_kv;
+    p.Tq = Tq;
+    p.Tk = Tk;
+    p.causal = causal;
+    p.rows = p.group * Tq;
+    p.nrb = g.nrb;
+    p.nkt = g.nkt;
+    p.balanced = g.balanced;
+    p.chunk = g.chunk;
+    p.splits = g.eff;
+    p.tot = g.tot;
+    p.G = g.G;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.limit_ns = kWaitLimitNs;
+    return p;
 }
 
 template <int D>
@@ -296,34 +351,36 @@ int launch_decode(const void *q, const void *k, const void *v, void *o, float *l
                   cudaStream_t stream, int sms)
 {
     using C = attn::DecCfg<D>;
-    int nkt, chunk, eff;
-    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, nkt, chunk, eff);
+    DecGeom g;
+    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, g);
     const long long nrows = (long long)B * H * Tq;
     CUtensorMap mq, mk, mv;
     if (make_map(&mq, q, D, (uint64_t)nrows, 1, 128) ||
         make_map(&mk, k, D, Tk, (uint64_t)B * H_kv, 128) ||
         make_map(&mv, v, D, Tk, (uint64_t)B * H_kv, 128))
         return ATTN_ERR_LAUNCH;
-    attn::DecodeParams p;
+    attn::DecodeParams p = decode_params(B, H, H_kv, Tq, Tk, causal, scale, g);
     p.part_o = static_cast<float *>(ws);
-    p.part_lse = p.part_o + (size_t)eff * nrows * D;
-    p.H = H;
-    p.H_kv = H_kv;
-    p.group = H / H_kv;
-    p.Tq = Tq;
-    p.Tk = Tk;
-    p.causal = causal;
-    p.rows = p.group * Tq;
-    p.nkt = nkt;
-    p.chunk = chunk;
-    p.splits = eff;
-    p.c_log2 = scale * 1.4426950408889634f;
-    p.limit_ns = kWaitLimitNs;
-    const dim3 grid(eff, B * H_kv, (p.rows + 127) / 128);
+    p.part_lse = p.part_o + (size_t)g.slots * nrows * D;
+    const dim3 grid = g.balanced ? dim3((unsigned)g.G, 1, 1) : dim3(g.eff, B * H_kv, g.nrb);
     attn::decode_partial_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
     if (launch_status()) return ATTN_ERR_LAUNCH;
-    attn::decode_combine_kernel<D><<<(unsigned)((nrows + 7) / 8), 256, 0, stream>>>(
-        p.part_o, p.part_lse, static_cast<__nv_bfloat16 *>(o), lse, nrows, eff);
+    // The merge is launched as a programmatic dependent of the partial kernel:
+    // its launch overlaps the partial kernel's tail and it waits on the device
+    // (griddepcontrol.wait) until every partial result is written.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((nrows + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn::decode_combine_kernel<D>, p,
+                           static_cast<__nv_bfloat16 *>(o), lse) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
     return launch_status();
 }
 
@@ -338,9 +395,9 @@ size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int d
         return 0;
     int sms = 0;
     if (splits <= 0 && device_ready(&sms)) return 0;
-    int nkt, chunk, eff;
-    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, nkt, chunk, eff);
-    return (size_t)eff * B * H * Tq * (size_t)(d_h + 1) * 4;
+    DecGeom g;
+    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, g);
+    return (size_t)g.slots * B * H * Tq * (size_t)(d_h + 1) * 4;
 }
 
 int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
@@ -352,6 +409,7 @@ int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float 
     if (!ws) return ATTN_ERR_NULL;
     if (misaligned(ws)) return ATTN_ERR_ALIGN;
     if (H_kv < 1 || H % H_kv != 0 || Tk < Tq || (long long)B * H_kv > 65535 ||
+        ((long long)(H / H_kv) * Tq + 127) / 128 > 65535 ||
         (long long)B * H * Tq > INT_MAX || (long long)B * H_kv * Tk > INT_MAX)
         return ATTN_ERR_BAD_SHAPE;
     int sms = 0;
@@ -567,6 +625,35 @@ int attn_selftest_set_mma_order(int mode)
 }
 
 int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
+
+int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms,
+                              int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots)
+{
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Tq < 1 || Tk < Tq || sms < 1 ||
+        (long long)B * H_kv > 65535 || (long long)B * H * Tq > INT_MAX)
+        return -1;
+    DecGeom g;
+    decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, g);
+    const attn::DecodeParams p = decode_params(B, H, H_kv, Tq, Tk, 1, 1.f, g);
+    const int gx = g.balanced ? g.G : g.eff, gy = g.balanced ? 1 : B * H_kv, gz = g.balanced ? 1 : g.nrb;
+    long long nrec = 0;
+    for (int bz = 0; bz < gz; ++bz)
+        for (int by = 0; by < gy; ++by)
+            for (int bx = 0; bx < gx; ++bx) {
+                attn::DecSeg sg;
+                for (int idx = 0; attn::dec_segment(p, bx, by, bz, idx, sg); ++idx, ++nrec) {
+                    if (!segs || nrec >= seg_cap) continue;
+                    int *r = segs + 8 * nrec;
+                    r[0] = bx; r[1] = by; r[2] = bz;
+                    r[3] = sg.kvbh; r[4] = sg.qt; r[5] = sg.t0; r[6] = sg.n; r[7] = sg.slot;
+                }
+            }
+    const long long W = (long long)B * H_kv * g.nrb;
+    for (long long w = 0; nseg && w < W && w < nseg_cap; ++w)
+        nseg[w] = g.balanced ? attn::dec_nseg(w, g.nkt, g.tot, g.G) : g.eff;
+    if (slots) *slots = g.slots;
+    return nrec > INT_MAX ? INT_MAX : (int)nrec;
+}
 
 int attn_selftest_set_exp_split(int pairs_of_8)
 {

@@ -85,14 +85,19 @@ int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *ls
  * "FlashAttention -- avoid writing the giant intermediate": persistent K/V
  * state in cached decoding, measured apart from prefill).  Grouped-query heads
  * as attn_fwd_gqa.  The key range is split across CTAs (split-KV) and the
- * splits' partial results are merged by their log-sum-exp.
+ * pieces' partial results are merged by their log-sum-exp.
  *   q, o   : bf16 [B, H, Tq, d_h];  k, v : bf16 [B, H_kv, Tk, d_h]
  *   lse    : out, fp32 [B, H, Tq]
  *   ws     : caller-owned device workspace of attn_decode_workspace_bytes()
  *            bytes for the same sizes and splits (partial outputs)
- *   splits : key splits (clamped to [1, ceil(Tk / 128)]); <= 0 picks enough
- *            for about two CTAs per SM
- * Other arguments, errors and asynchrony as attn_fwd.
+ *   splits : > 0: every head's keys cut into that many equal ranges (clamped
+ *            to [1, ceil(Tk / 128)]), one CTA each;  < 0: balanced -- one CTA
+ *            per SM, all heads' 128-key tiles dealt out in equal contiguous
+ *            ranges (a head may span several CTAs, a CTA several heads);
+ *            0: automatic -- the split that fills one wave of one CTA per SM
+ *            when that keeps at least 85 % of the SMs busy, else balanced
+ * (H / H_kv) * Tq <= 65535 * 128.  Other arguments, errors and asynchrony as
+ * attn_fwd.
  */
 int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
                     int B, int H, int H_kv, int Tq, int Tk, int d_h, int causal, float scale,

@@ -40,6 +40,16 @@ def _case(B, H, H_kv, Tq, Tk, D, causal, splits, seed):
     (1, 32, 8, 64, 2048, 128, True, 4),
     (3, 6, 3, 5, 333, 128, True, 2),
     (1, 2, 1, 1, 1, 64, True, 0),
+    # balanced partition (splits < 0): one head over 128 CTAs of one tile each
+    (1, 2, 1, 1, 16384, 128, True, -1),
+    # 512 heads of 4 tiles over the SMs: several heads (segments) per CTA
+    (64, 8, 8, 1, 512, 64, True, -1),
+    (64, 8, 8, 1, 512, 64, True, 0),
+    # three blocks of packed rows per K/V head (8 x 40 = 320 rows), 6 tiles each
+    (2, 32, 4, 40, 700, 128, True, -1),
+    (2, 32, 4, 40, 700, 128, True, 0),
+    (3, 12, 4, 7, 5000, 128, False, -1),
+    (3, 12, 4, 7, 5000, 128, False, 0),
 ])
 def test_decode_every_element(B, H, H_kv, Tq, Tk, D, causal, splits):
     st = _case(B, H, H_kv, Tq, Tk, D, causal, splits, 7700 + Tq + Tk + D + splits)
