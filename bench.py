@@ -69,7 +69,12 @@ def parse():
     ap.add_argument("--exp-split", type=int, default=None,
                     help="fused kernel variant: column pairs of every 8 whose exponentials run "
                          "on the FMA pipe (0, 2, 3, 4); default: the library's choice")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.e2e_steps < 1 or args.steps < 1:
+        ap.error("--steps and --e2e-steps must be at least 1")
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    return args
 
 
 def workload_of(args):
