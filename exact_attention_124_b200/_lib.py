@@ -62,7 +62,7 @@ def load_library():
     lib.attn_selftest_set_mma_order.argtypes = [I]
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
-    lib.attn_selftest_decode_plan.argtypes = [I, I, I, I, I, I, I, P, I, P, I, P]
+    lib.attn_selftest_decode_plan.argtypes = [I, I, I, I, I, I, I, P, I, P, I, P, P]
     for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_decode", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
@@ -268,23 +268,25 @@ def set_exp_split(pairs_of_8: int) -> int:
 
 def decode_plan(B: int, H: int, H_kv: int, Tq: int, Tk: int, splits: int, sms: int):
     """Host-side work plan of attn_fwd_decode on a device with ``sms`` SMs
-    (no device needed): (segments, nseg, slots) with segments a list of
-    (cta_x, cta_y, cta_z, kvbh, row_block, first_tile, tiles, slot) tuples and
+    (no device needed): (segments, nseg, slots, copies) with segments a list of
+    (cta_x, cta_y, cta_z, kvbh, row_block, first_tile, tiles, first_slot)
+    tuples (a segment fills slots first_slot .. first_slot + copies - 1) and
     nseg[w] the partial slots the merge reads for head w."""
     lib = load_library()
     nrb = ((H // H_kv) * Tq + 127) // 128 if H_kv > 0 and H % H_kv == 0 else 0
     heads = B * H_kv * nrb
-    slots = ctypes.c_int(0)
+    slots, copies = ctypes.c_int(0), ctypes.c_int(0)
     n = lib.attn_selftest_decode_plan(B, H, H_kv, Tq, Tk, splits, sms, None, 0, None, 0,
-                                      ctypes.byref(slots))
+                                      ctypes.byref(slots), ctypes.byref(copies))
     if n < 0:
         raise ValueError("bad decode sizes")
     segs = (ctypes.c_int * (8 * max(n, 1)))()
     nseg = (ctypes.c_int * max(heads, 1))()
     n2 = lib.attn_selftest_decode_plan(B, H, H_kv, Tq, Tk, splits, sms, segs, n, nseg, heads,
-                                       ctypes.byref(slots))
+                                       ctypes.byref(slots), ctypes.byref(copies))
     assert n2 == n
-    return ([tuple(segs[8 * i:8 * i + 8]) for i in range(n)], list(nseg[:heads]), slots.value)
+    return ([tuple(segs[8 * i:8 * i + 8]) for i in range(n)], list(nseg[:heads]), slots.value,
+            copies.value)
 
 
 def fused_grid_ctas(B: int, H: int, T: int, D: int, causal: bool) -> int:

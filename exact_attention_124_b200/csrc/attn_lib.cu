@@ -103,8 +103,12 @@ int device_ready(int *sms_out)
         ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<64>, attn::BwdCfg<64>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<128>, attn::BwdCfg<128>::SMEM);
-        ok &= set_smem(attn::decode_partial_kernel<64>, attn::DecCfg<64>::SMEM);
-        ok &= set_smem(attn::decode_partial_kernel<128>, attn::DecCfg<128>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<64, 1>, attn::DecCfg<64>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<64, 2>, attn::DecCfg<64>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<64, 4>, attn::DecCfg<64>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<128, 1>, attn::DecCfg<128>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<128, 2>, attn::DecCfg<128>::SMEM);
+        ok &= set_smem(attn::decode_partial_kernel<128, 4>, attn::DecCfg<128>::SMEM);
         ok &= fused_all_ready<64>();
         ok &= fused_all_ready<128>();
         ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
@@ -280,6 +284,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 // enough splits for about two CTAs per SM.
 struct DecGeom {
     int nkt, nrb, balanced, chunk, eff, G, slots;
+    int copies;  // copies of the packed rows in the 128-row tile (4, 2 or 1)
     long long tot;
 };
 
@@ -291,7 +296,9 @@ struct DecGeom {
 void decode_geometry(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms, DecGeom &g)
 {
     g.nkt = (Tk + 127) / 128;
-    g.nrb = ((H / H_kv) * Tq + 127) / 128;
+    const long long rows = (long long)(H / H_kv) * Tq;  // packed rows per K/V head
+    g.copies = rows <= 32 ? 4 : rows <= 64 ? 2 : 1;
+    g.nrb = (int)((rows + 127) / 128);
     g.tot = (long long)B * H_kv * g.nrb * g.nkt;
     const long long heads = (long long)B * H_kv * g.nrb;
     if (splits == 0) {
@@ -335,6 +342,7 @@ attn::DecodeParams decode_params(int B, int H, int H_kv, int Tq, int Tk, int cau
     p.rows = p.group * Tq;
     p.nrb = g.nrb;
     p.nkt = g.nkt;
+    p.copies = g.copies;
     p.balanced = g.balanced;
     p.chunk = g.chunk;
     p.splits = g.eff;
@@ -355,15 +363,21 @@ int launch_decode(const void *q, const void *k, const void *v, void *o, float *l
     decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, g);
     const long long nrows = (long long)B * H * Tq;
     CUtensorMap mq, mk, mv;
-    if (make_map(&mq, q, D, (uint64_t)nrows, 1, 128) ||
+    // the Q box is one copy of the rows: 128 / copies rows
+    if (make_map(&mq, q, D, (uint64_t)nrows, 1, 128 / g.copies) ||
         make_map(&mk, k, D, Tk, (uint64_t)B * H_kv, 128) ||
         make_map(&mv, v, D, Tk, (uint64_t)B * H_kv, 128))
         return ATTN_ERR_LAUNCH;
     attn::DecodeParams p = decode_params(B, H, H_kv, Tq, Tk, causal, scale, g);
     p.part_o = static_cast<float *>(ws);
-    p.part_lse = p.part_o + (size_t)g.slots * nrows * D;
+    p.part_lse = p.part_o + (size_t)g.slots * g.copies * nrows * D;
     const dim3 grid = g.balanced ? dim3((unsigned)g.G, 1, 1) : dim3(g.eff, B * H_kv, g.nrb);
-    attn::decode_partial_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    if (g.copies == 4)
+        attn::decode_partial_kernel<D, 4><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    else if (g.copies == 2)
+        attn::decode_partial_kernel<D, 2><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    else
+        attn::decode_partial_kernel<D, 1><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
     if (launch_status()) return ATTN_ERR_LAUNCH;
     // The merge is launched as a programmatic dependent of the partial kernel:
     // its launch overlaps the partial kernel's tail and it waits on the device
@@ -397,7 +411,7 @@ size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int d
     if (splits <= 0 && device_ready(&sms)) return 0;
     DecGeom g;
     decode_geometry(B, H, H_kv, Tq, Tk, splits, sms, g);
-    return (size_t)g.slots * B * H * Tq * (size_t)(d_h + 1) * 4;
+    return (size_t)g.slots * g.copies * B * H * Tq * (size_t)(d_h + 1) * 4;
 }
 
 int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, void *ws,
@@ -627,7 +641,8 @@ int attn_selftest_set_mma_order(int mode)
 int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
 
 int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms,
-                              int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots)
+                              int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots,
+                              int *copies)
 {
     if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Tq < 1 || Tk < Tq || sms < 1 ||
         (long long)B * H_kv > 65535 || (long long)B * H * Tq > INT_MAX)
@@ -645,13 +660,14 @@ int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits
                     if (!segs || nrec >= seg_cap) continue;
                     int *r = segs + 8 * nrec;
                     r[0] = bx; r[1] = by; r[2] = bz;
-                    r[3] = sg.kvbh; r[4] = sg.qt; r[5] = sg.t0; r[6] = sg.n; r[7] = sg.slot;
+                    r[3] = sg.kvbh; r[4] = sg.qt; r[5] = sg.t0; r[6] = sg.n; r[7] = sg.slot * g.copies;
                 }
             }
     const long long W = (long long)B * H_kv * g.nrb;
     for (long long w = 0; nseg && w < W && w < nseg_cap; ++w)
-        nseg[w] = g.balanced ? attn::dec_nseg(w, g.nkt, g.tot, g.G) : g.eff;
-    if (slots) *slots = g.slots;
+        nseg[w] = (g.balanced ? attn::dec_nseg(w, g.nkt, g.tot, g.G) : g.eff) * g.copies;
+    if (slots) *slots = g.slots * g.copies;
+    if (copies) *copies = g.copies;
     return nrec > INT_MAX ? INT_MAX : (int)nrec;
 }
 

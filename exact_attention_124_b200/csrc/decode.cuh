@@ -16,7 +16,14 @@
 //   fixed:   every head cut into `splits` equal key ranges, one CTA each.
 //   decode_partial_kernel  the rows packed into the M = 128 tile are (query
 //                          head of the K/V head's group, query) pairs, so a
-//                          grouped-query group shares each K/V tile.  Online
+//                          grouped-query group shares each K/V tile.  With
+//                          R = group * Tq <= 32 (64) real rows, the tile holds
+//                          CP = 4 (2) copies of them, one per 128 / CP lanes,
+//                          and copy c takes only keys [c W, c W + W) of every
+//                          tile (W = 128 / CP; P is zero elsewhere in its
+//                          rows): each softmax thread does W instead of 128
+//                          exponentials and the copies are merged like
+//                          further key splits.  Online
 //                          softmax over a segment's tiles exactly as the
 //                          prefill kernel (S = Q K^T and O += P V on tcgen05, S
 //                          double buffered in TMEM so the next score tile is
@@ -40,6 +47,7 @@ struct DecodeParams {
     int rows;         // packed query rows per K/V head: group * Tq
     int nrb;          // blocks of 128 packed rows per K/V head
     int nkt;          // key tiles of 128
+    int copies;       // CP: copies of the packed rows in the 128-row tile
     int balanced;     // 1: balanced ranges over G CTAs; 0: fixed splits
     int chunk;        // fixed: key tiles per split
     int splits;       // fixed: splits per head (= partial slots)
@@ -112,7 +120,7 @@ struct DecCfg {
     static constexpr int OFF_Q = 0;                // [2] Q tiles
     static constexpr int OFF_KV = 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 2 + 1 + 1 + 1;
+    static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 2 + 1 + 1 + 1 + 1;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
     static constexpr int THREADS = 192;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -122,7 +130,7 @@ struct DecCfg {
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
 };
 
-template <int D>
+template <int D, int CP>
 __global__ void __launch_bounds__(192, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -143,8 +151,14 @@ __global__ void __launch_bounds__(192, 1)
     // one P barrier per S buffer: a single one could complete twice (two
     // tiles) before the MMA warp waits on the first, aliasing its phase
     const uint32_t b_pfull = b_sfull + 16;  // [2]
+    // b_pvdone completes after every P V (the lazy rescale waits for the
+    // previous one: only that one can be outstanding there).  The epilogue
+    // waits on b_pvlast, completed once per segment after its last P V: with
+    // the per-tile barrier the last P V's parity could alias the one before
+    // it while both are still in flight.
     const uint32_t b_pvdone = b_pfull + 16;
-    const uint32_t b_ofree = b_pvdone + 8;  // the softmax warps have read a segment's O
+    const uint32_t b_pvlast = b_pvdone + 8;
+    const uint32_t b_ofree = b_pvlast + 8;  // the softmax warps have read a segment's O
     const uint32_t b_drain = b_ofree + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -163,6 +177,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(b_kvempty + 8 * s, 1);
         }
         mbar_init(b_pvdone, 1);
+        mbar_init(b_pvlast, 1);
         mbar_init(b_ofree, 128);
         mbar_init(b_drain, 1);
         *abort_flag = 0;
@@ -195,9 +210,12 @@ __global__ void __launch_bounds__(192, 1)
                 qarmed_par = (qarmed_par & ~(1u << qb)) | (qpar << qb);
                 const int b = sg.kvbh / p.H_kv, kvl = sg.kvbh % p.H_kv;
                 const int qrow0 = (b * p.H + kvl * p.group) * p.Tq + sg.qt * 128;
+                // CP copies of the R = 128 / CP rows (the map's box is R rows)
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sQ + qb * C::TILE + kb * C::SUB, &tmQ, b_qfull + 8 * qb, 64 * kb, qrow0,
-                                0, pol_q);
+#pragma unroll
+                    for (int cp = 0; cp < CP; ++cp)
+                        tma_load_3d(sQ + qb * C::TILE + kb * C::SUB + cp * (128 / CP) * 128, &tmQ,
+                                    b_qfull + 8 * qb, 64 * kb, qrow0, 0, pol_q);
                 auto load = [&](const CUtensorMap *map, int tile) -> bool {
                     if (!mbar_wait(b_kvempty + 8 * idx, ph ^ 1u, lim, W_D_KVEMPTY, abort_flag)) return false;
                     mbar_arrive_expect_tx(b_kvfull + 8 * idx, C::TILE);
@@ -280,6 +298,7 @@ __global__ void __launch_bounds__(192, 1)
                                sw128_desc_join(vl + kk * (2048 >> 4), 1024), C::IDESC_PV,
                                (j > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(b_pvdone);
+                    if (j == n - 1) tc_commit(b_pvlast);
                     tc_commit(b_kvempty + 8 * vs);
                     if (j + 2 < n) {  // the next score tile into the buffer just consumed
                         if (!(ok = next(slot))) break;
@@ -296,8 +315,10 @@ __global__ void __launch_bounds__(192, 1)
                 mbar_wait(b_drain, 0, lim, W_D_DRAIN);
             }
         }
-    } else if (warp < 4) {  // softmax: thread = packed query row
+    } else if (warp < 4) {  // softmax: thread = packed query row of one copy
+        constexpr int W = 128 / CP;  // rows per copy, and keys per copy in each tile
         const int r = warp * 32 + lane;
+        const int cp = r / W, rr = r % W;  // copy (warp-uniform), row within the copy
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const float cl2 = p.c_log2;
         bool ok = true;
@@ -305,7 +326,7 @@ __global__ void __launch_bounds__(192, 1)
         DecSeg sg;
         for (int si = 0; ok && dec_segment(p, blockIdx.x, blockIdx.y, blockIdx.z, si, sg); ++si) {
             const int n = sg.n;
-            const int pr = sg.qt * 128 + r;
+            const int pr = sg.qt * 128 + rr;
             const bool valid = pr < p.rows;
             const int g = valid ? pr / p.Tq : 0, qi = valid ? pr % p.Tq : 0;
             const int pos = p.Tk - p.Tq + qi;
@@ -318,24 +339,33 @@ __global__ void __launch_bounds__(192, 1)
                 if (!(ok = __all_sync(0xffffffffu, w))) break;
                 tc_fence_after_sync();
                 const uint32_t tS = tmem + lane_off + C::TM_S + 128 * buf;
-                float s[128];
-                {
-                    uint32_t rr[128];
-                    tmem_ld128(tS, rr);
-                    tmem_wait_ld_regs128(rr);
+                float s[W];
+                if constexpr (W == 128) {
+                    uint32_t rg[128];
+                    tmem_ld128(tS, rg);
+                    tmem_wait_ld_regs128(rg);
 #pragma unroll
-                    for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(rr[i]);
+                    for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(rg[i]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < W / 32; ++c) {
+                        uint32_t rg[32];
+                        tmem_ld32(tS + cp * W + 32 * c, rg);
+                        tmem_wait_ld_regs(rg);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rg[i]);
+                    }
                 }
-                const int key0 = 128 * (sg.t0 + j);
-                const bool need_mask = (key0 + 128 > p.Tk) || (p.causal && key0 + 127 > p.Tk - p.Tq);
+                const int key0 = 128 * (sg.t0 + j) + cp * W;  // key of s[0]
+                const bool need_mask = (key0 + W > p.Tk) || (p.causal && key0 + W - 1 > p.Tk - p.Tq);
                 if (need_mask) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
+                    for (int c = 0; c < W; ++c)
                         if (key0 + c > lim_key) s[c] = -INFINITY;
                 }
                 float mx = s[0];
 #pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+                for (int c = 1; c < W; ++c) mx = fmaxf(mx, s[c]);
                 const float cand = mx * cl2;
                 float alpha = 1.f;
                 bool resc = false;
@@ -352,28 +382,44 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after_sync();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
-                        uint32_t rr[32];
-                        tmem_ld32(tmem + lane_off + C::TM_O + 32 * c, rr);
-                        tmem_wait_ld_regs(rr);
+                        uint32_t rg[32];
+                        tmem_ld32(tmem + lane_off + C::TM_O + 32 * c, rg);
+                        tmem_wait_ld_regs(rg);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-                        tmem_st32(tmem + lane_off + C::TM_O + 32 * c, rr);
+                        for (int i = 0; i < 32; ++i) rg[i] = __float_as_uint(__uint_as_float(rg[i]) * alpha);
+                        tmem_st32(tmem + lane_off + C::TM_O + 32 * c, rg);
                     }
                 }
                 l *= alpha;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 float ls = 0.f;
+                // P over the first 64 S columns (bf16 pairs): this copy's W keys
+                // at pair columns [cp W / 2, cp W / 2 + W / 2), zeros elsewhere
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[32];
+                for (int h = 0; h < (W + 63) / 64; ++h) {
+                    constexpr int NP = W < 64 ? W / 2 : 32;  // pairs in this store
+                    uint32_t pk[NP];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < NP; ++i) {
                         const float p0 = fast_exp2(fmaf(s[64 * h + 2 * i], cl2, neg_m));
                         const float p1 = fast_exp2(fmaf(s[64 * h + 2 * i + 1], cl2, neg_m));
                         ls += p0 + p1;
                         pk[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(tS + 32 * h, pk);
+                    if constexpr (NP == 32) tmem_st32(tS + cp * (W / 2) + 32 * h, pk);
+                    else tmem_st16(tS + cp * (W / 2), pk);
+                }
+                if constexpr (CP == 2) {
+                    uint32_t z[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) z[i] = 0u;
+                    tmem_st32(tS + (1 - cp) * 32, z);
+                } else if constexpr (CP == 4) {
+                    uint32_t z[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+                    for (int o = 1; o < 4; ++o) tmem_st16(tS + ((cp + o) & 3) * 16, z);
                 }
                 l += ls;
                 tmem_wait_st();
@@ -382,24 +428,25 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (!ok) break;
             u += n;
-            const bool w = mbar_wait(b_pvdone, (u - 1) & 1u, lim, W_D_PVDONE, abort_flag);
+            const bool w = mbar_wait(b_pvlast, (uint32_t)si & 1u, lim, W_D_PVDONE, abort_flag);
             if (!(ok = __all_sync(0xffffffffu, w))) break;
             tc_fence_after_sync();
             const int b = sg.kvbh / p.H_kv, kvl = sg.kvbh % p.H_kv;
             const size_t row = (size_t)(b * p.H + kvl * p.group + g) * p.Tq + qi;
-            const size_t at = (size_t)sg.slot * (size_t)p.nrows + row;
+            // each copy's result is one more partial of this row
+            const size_t at = ((size_t)sg.slot * CP + cp) * (size_t)p.nrows + row;
             const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(tmem + lane_off + C::TM_O + 32 * c, rr);
-                tmem_wait_ld_regs(rr);
+                uint32_t rg[32];
+                tmem_ld32(tmem + lane_off + C::TM_O + 32 * c, rg);
+                tmem_wait_ld_regs(rg);
                 if (valid) {
                     float4 *dst = reinterpret_cast<float4 *>(p.part_o + at * D + 32 * c);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(rr[4 * i]) * inv, __uint_as_float(rr[4 * i + 1]) * inv,
-                                             __uint_as_float(rr[4 * i + 2]) * inv, __uint_as_float(rr[4 * i + 3]) * inv);
+                        dst[i] = make_float4(__uint_as_float(rg[4 * i]) * inv, __uint_as_float(rg[4 * i + 1]) * inv,
+                                             __uint_as_float(rg[4 * i + 2]) * inv, __uint_as_float(rg[4 * i + 3]) * inv);
                 }
             }
             tc_fence_before_sync();
@@ -435,6 +482,7 @@ __global__ void __launch_bounds__(256)
         const long long w = (b * p.H_kv + h / p.group) * p.nrb + pr / 128;
         splits = dec_nseg(w, p.nkt, p.tot, p.G);
     }
+    splits *= p.copies;  // every segment wrote one partial per copy of the rows
     float mx = -INFINITY;
     for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[(size_t)s * nrows + r]);
     constexpr int PER = D / 32;

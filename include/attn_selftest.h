@@ -76,17 +76,20 @@ int attn_selftest_last_wait_site(void);
  * for these sizes and `splits` on a device with `sms` SMs, computed by the
  * same code the kernel runs.  A head is (batch * H_kv + K/V head, block of 128
  * packed query rows), numbered w = kvbh * ceil((H / H_kv) * Tq / 128) + block.
- *   segs  : up to seg_cap records of 8 ints
- *           (cta.x, cta.y, cta.z, kvbh, row block, first key tile, tiles, slot)
- *           -- one per segment, a segment being one head's key tiles in one CTA,
- *           its partial result going to partial slot `slot` of that head
- *   nseg  : for heads w < nseg_cap, how many partial slots the merge reads
- *   slots : the workspace's partial slots per query row
+ *   segs   : up to seg_cap records of 8 ints
+ *            (cta.x, cta.y, cta.z, kvbh, row block, first key tile, tiles, slot)
+ *            -- one per segment, a segment being one head's key tiles in one
+ *            CTA, its partial results going to partial slots slot .. slot +
+ *            copies - 1 of that head (one per copy of the packed rows)
+ *   nseg   : for heads w < nseg_cap, how many partial slots the merge reads
+ *   slots  : the workspace's partial slots per query row
+ *   copies : copies of the packed query rows in the 128-row tile (4, 2, 1)
  * Returns the number of segments (records beyond seg_cap are not written),
  * or -1 for bad sizes.
  */
 int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms,
-                              int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots);
+                              int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots,
+                              int *copies);
 
 #ifdef __cplusplus
 }

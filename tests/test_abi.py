@@ -133,4 +133,7 @@ def test_decode_rejects_bad_arguments(lib):
     bad = list(ok); bad[8] = 3               # 8 heads over 3 K/V heads
     assert lib.attn_fwd_decode(*bad) == 3
     # workspace size with explicit splits needs no device: 4 splits x rows x (d + 1) floats
-    assert lib.attn_decode_workspace_bytes(1, 8, 2, 4, 1024, 128, 4) == 4 * 1 * 8 * 4 * 129 * 4
+    # 4 splits x 4 copies of the 16 packed rows (group 4 x Tq 4), B*H*Tq rows of (d_h + 1) floats
+    assert lib.attn_decode_workspace_bytes(1, 8, 2, 4, 1024, 128, 4) == 4 * 4 * 1 * 8 * 4 * 129 * 4
+    # 80 packed rows (group 4 x Tq 20): one copy
+    assert lib.attn_decode_workspace_bytes(1, 8, 2, 20, 1024, 128, 4) == 4 * 1 * 8 * 20 * 129 * 4

@@ -1,8 +1,9 @@
 """The decode work plan (attn_selftest_decode_plan: the library's own host and
 kernel partition code run on the CPU) covers every (head, key tile) exactly
 once, gives every head's partial slots 0 .. nseg-1 exactly once (the slots the
-merge kernel reads), stays inside the workspace's slot count, and in balanced
-mode deals the same number of tiles (within one) to every CTA."""
+merge kernel reads; a segment fills one slot per copy of the packed rows),
+stays inside the workspace's slot count, and in balanced mode deals the same
+number of tiles (within one) to every CTA."""
 import itertools
 import random
 from collections import Counter, defaultdict
@@ -13,9 +14,11 @@ import exact_attention_124_b200 as attn
 
 
 def _check(B, H, H_kv, Tq, Tk, splits, sms):
-    segs, nseg, slots = attn.decode_plan(B, H, H_kv, Tq, Tk, splits, sms)
+    segs, nseg, slots, copies = attn.decode_plan(B, H, H_kv, Tq, Tk, splits, sms)
     nkt = (Tk + 127) // 128
-    nrb = ((H // H_kv) * Tq + 127) // 128
+    rows = (H // H_kv) * Tq
+    nrb = (rows + 127) // 128
+    assert copies == (4 if rows <= 32 else 2 if rows <= 64 else 1)
     heads = B * H_kv * nrb
     assert len(nseg) == heads
     covered = Counter()
@@ -28,10 +31,10 @@ def _check(B, H, H_kv, Tq, Tk, splits, sms):
         w = kvbh * nrb + qt
         for t in range(t0, t0 + n):
             covered[(w, t)] += 1
-        head_slots[w].append(slot)
+        head_slots[w].extend(range(slot, slot + copies))
         per_cta[(bx, by, bz)] += n
         ctas.add((bx, by, bz))
-        assert 0 <= slot < slots
+        assert 0 <= slot and slot + copies <= slots
     assert len(covered) == heads * nkt and set(covered.values()) == {1}
     for w in range(heads):
         assert sorted(head_slots[w]) == list(range(nseg[w])), (w, head_slots[w], nseg[w])
@@ -42,7 +45,7 @@ def _check(B, H, H_kv, Tq, Tk, splits, sms):
         s = min(splits, nkt)
         chunk = -(-nkt // s)
         assert len(ctas) == heads * (-(-nkt // chunk))
-    return segs, nseg, slots, len(ctas)
+    return segs, nseg, slots, len(ctas), copies
 
 
 SHAPES = [(2, 8, 2, 1, 4096), (1, 4, 4, 16, 1000), (1, 32, 8, 64, 2048), (3, 6, 3, 5, 333),
@@ -69,18 +72,19 @@ def test_decode_plan_random_shapes():
 
 def test_decode_plan_automatic_choice():
     # 32 heads of 64 tiles: 4 splits fill 128 of 148 SMs (86 %) in one wave
-    segs, _, _, ctas = _check(4, 32, 8, 1, 8192, 0, 148)
+    segs, _, _, ctas, copies = _check(4, 32, 8, 1, 8192, 0, 148)
     assert ctas == 128 and all(n == 16 for *_, n, _s in segs)
+    assert copies == 4  # group 4 x Tq 1 = 4 rows: four copies, 32 keys of every tile each
     # 100 heads: one wave of fixed splits would leave a third of the SMs idle -> balanced
-    segs, _, _, ctas = _check(100, 8, 8, 1, 8192, 0, 148)
+    segs, _, _, ctas, _ = _check(100, 8, 8, 1, 8192, 0, 148)
     assert ctas == 148 and all(c[1:3] == (0, 0) for c in segs)
 
 
 def test_decode_plan_balanced_spans_heads_and_ctas():
     # one head over 128 CTAs of one tile each, and 512 short heads over 148 CTAs
-    segs, nseg, _, _ = _check(1, 2, 1, 1, 16384, -1, 148)
-    assert nseg == [128]
-    segs, nseg, _, _ = _check(64, 8, 8, 1, 512, -1, 148)
+    segs, nseg, _, _, copies = _check(1, 2, 1, 1, 16384, -1, 148)
+    assert nseg == [128 * copies]
+    segs, nseg, _, _, _ = _check(64, 8, 8, 1, 512, -1, 148)
     per_cta = Counter(s[0] for s in segs)
     assert max(per_cta.values()) >= 4  # several heads (segments) in one CTA
 

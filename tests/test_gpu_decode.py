@@ -1,7 +1,9 @@
 """Parity of the split-KV decode path (attn_fwd_decode) with the float64
 oracle: Tq new queries against a Tk-token K/V cache, query i at position
 Tk - Tq + i ("FlashAttention -- avoid writing the giant intermediate": the
-persistent K/V state of cached decoding).  Same bounds as the prefill path."""
+persistent K/V state of cached decoding).  Same bounds as the prefill path.
+The cases cover fixed, balanced and automatic partitions and 1, 2 and 4
+copies of the packed query rows (more than 64, 33-64 and at most 32 rows)."""
 import math
 
 import numpy as np
@@ -50,6 +52,10 @@ def _case(B, H, H_kv, Tq, Tk, D, causal, splits, seed):
     (2, 32, 4, 40, 700, 128, True, 0),
     (3, 12, 4, 7, 5000, 128, False, -1),
     (3, 12, 4, 7, 5000, 128, False, 0),
+    # 33-64 packed rows: two copies of the rows, 64 keys of every tile each
+    (2, 8, 2, 12, 3000, 128, True, 0),
+    (1, 16, 2, 5, 900, 64, False, -1),
+    (1, 16, 2, 8, 260, 64, True, 3),
 ])
 def test_decode_every_element(B, H, H_kv, Tq, Tk, D, causal, splits):
     st = _case(B, H, H_kv, Tq, Tk, D, causal, splits, 7700 + Tq + Tk + D + splits)
