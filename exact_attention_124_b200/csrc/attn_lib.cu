@@ -35,6 +35,38 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// attn_fwd_host's copy pipeline: two non-blocking streams (host -> device,
+// device -> host) and events per chunk, created on first use per device.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t loaded[kHostChunks] = {}, computed[kHostChunks] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
+HostPipe *host_pipe()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostPipe &hp = g_pipe[dev];
+    if (hp.ready) return &hp;
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; ok && c < kHostChunks; ++c)
+        ok = cudaEventCreateWithFlags(&hp.loaded[c], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.computed[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    hp.ready = true;
+    return &hp;
+}
+
 int get_encoder()
 {
     if (g_encode) return ATTN_OK;
@@ -515,18 +547,57 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, vo
     int rc = validate(dq, dk, dv, do_, dlse, B, H, T, d_h, causal, scale);
     if (rc) return rc;
     if ((rc = device_ready(nullptr))) return rc;
+    HostPipe *hp = host_pipe();
+    if (!hp) return ATTN_ERR_LAUNCH;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t n = (size_t)B * H * T * d_h * 2;
-    const size_t nl = (size_t)B * H * T * sizeof(float);
-    if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return ATTN_ERR_LAUNCH;
+    // Heads are independent: cut the B * H heads into chunks and overlap the
+    // host -> device copy of chunk c + 1, the attention of chunk c (on
+    // `stream`) and the device -> host copy of chunk c - 1 (the two copy
+    // directions run on separate copy engines).
+    const int bh = B * H;
+    const int nch = bh < kHostChunks ? bh : kHostChunks;
+    const int per = (bh + nch - 1) / nch;
+    const size_t head = (size_t)T * d_h;  // elements of one head
+    auto cp = [](void *dst, const void *src, size_t bytes, cudaMemcpyKind kind, cudaStream_t st) {
+        return cudaMemcpyAsync(dst, src, bytes, kind, st) == cudaSuccess;
+    };
+    bool ok = cudaEventRecord(hp->start, s) == cudaSuccess &&  // earlier work on the buffers
+              cudaStreamWaitEvent(hp->in, hp->start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(hp->out, hp->start, 0) == cudaSuccess;
+    for (int c = 0; ok && c < nch; ++c) {
+        const int h0 = c * per, nh = (h0 + per <= bh ? per : bh - h0);
+        if (nh <= 0) break;
+        const size_t off = (size_t)h0 * head * 2, bytes = (size_t)nh * head * 2;
+        ok = cp(static_cast<char *>(dq) + off, static_cast<const char *>(q_host) + off, bytes,
+                cudaMemcpyHostToDevice, hp->in) &&
+             cp(static_cast<char *>(dk) + off, static_cast<const char *>(k_host) + off, bytes,
+                cudaMemcpyHostToDevice, hp->in) &&
+             cp(static_cast<char *>(dv) + off, static_cast<const char *>(v_host) + off, bytes,
+                cudaMemcpyHostToDevice, hp->in) &&
+             cudaEventRecord(hp->loaded[c], hp->in) == cudaSuccess;
     }
-    if ((rc = attn_fwd(dq, dk, dv, do_, dlse, B, H, T, d_h, causal, scale, stream))) return rc;
-    if (cudaMemcpyAsync(o_host, do_, n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse_host, dlse, nl, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    for (int c = 0; ok && c < nch; ++c) {
+        const int h0 = c * per, nh = (h0 + per <= bh ? per : bh - h0);
+        if (nh <= 0) break;
+        const size_t off = (size_t)h0 * head * 2, bytes = (size_t)nh * head * 2;
+        const size_t loff = (size_t)h0 * T * sizeof(float), lbytes = (size_t)nh * T * sizeof(float);
+        if (!(ok = cudaStreamWaitEvent(s, hp->loaded[c], 0) == cudaSuccess)) break;
+        if ((rc = attn_fwd(static_cast<const char *>(dq) + off, static_cast<const char *>(dk) + off,
+                           static_cast<const char *>(dv) + off, static_cast<char *>(do_) + off,
+                           reinterpret_cast<float *>(reinterpret_cast<char *>(dlse) + loff), 1, nh,
+                           T, d_h, causal, scale, stream)))
+            return rc;
+        ok = cudaEventRecord(hp->computed[c], s) == cudaSuccess &&
+             cudaStreamWaitEvent(hp->out, hp->computed[c], 0) == cudaSuccess &&
+             cp(static_cast<char *>(o_host) + off, static_cast<const char *>(do_) + off, bytes,
+                cudaMemcpyDeviceToHost, hp->out) &&
+             cp(reinterpret_cast<char *>(lse_host) + loff, reinterpret_cast<const char *>(dlse) + loff,
+                lbytes, cudaMemcpyDeviceToHost, hp->out);
+    }
+    // `stream` completes only after the last copy back
+    ok = ok && cudaEventRecord(hp->done, hp->out) == cudaSuccess &&
+         cudaStreamWaitEvent(s, hp->done, 0) == cudaSuccess;
+    if (!ok) {
         (void)cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }

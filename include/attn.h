@@ -175,9 +175,15 @@ int attn_fwd_unfused_noalloc(const void *q, const void *k, const void *v, void *
 /*
  * Fused forward with HOST buffers: copies q/k/v host -> device into the
  * caller's device buffers dq/dk/dv, runs attn_fwd into do_/dlse, and copies
- * O and lse back to o_host/lse_host, all in order on `stream`.  Host buffers
- * should be pinned (cudaHostAlloc) for asynchronous copies.  The call returns
- * once everything is enqueued; synchronise `stream` before reading o_host.
+ * O and lse back to o_host/lse_host.  The B * H heads are cut into up to 8
+ * chunks so that the host -> device copy of one chunk, the attention of the
+ * previous one (on `stream`) and the copy back of the one before run at the
+ * same time (two library-owned streams, created on the first call per
+ * device, carry the copies; they wait for the work already on `stream` and
+ * `stream` waits for them at the end).  Host buffers should be pinned
+ * (cudaHostAlloc) for asynchronous copies.  The call returns once everything
+ * is enqueued; synchronise `stream` before reading o_host.  Not for
+ * concurrent use from several host threads.
  */
 int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
                   float *lse_host, void *dq, void *dk, void *dv, void *do_, float *dlse, int B,
