@@ -133,8 +133,8 @@ int device_ready(int *sms_out)
         bool ok = true;
         ok &= set_smem(attn::bwd_dkdv_kernel<64>, attn::BwdCfg<64>::SMEM);
         ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
-        ok &= set_smem(attn::bwd_dq_kernel<64>, attn::BwdCfg<64>::SMEM);
-        ok &= set_smem(attn::bwd_dq_kernel<128>, attn::BwdCfg<128>::SMEM);
+        ok &= set_smem(attn::bwd_dq_kernel<64>, attn::DqCfg<64>::SMEM);
+        ok &= set_smem(attn::bwd_dq_kernel<128>, attn::DqCfg<128>::SMEM);
         ok &= set_smem(attn::decode_partial_kernel<64, 1>, attn::DecCfg<64>::SMEM);
         ok &= set_smem(attn::decode_partial_kernel<64, 2>, attn::DecCfg<64>::SMEM);
         ok &= set_smem(attn::decode_partial_kernel<64, 4>, attn::DecCfg<64>::SMEM);
@@ -307,13 +307,12 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     if (launch_status()) return ATTN_ERR_LAUNCH;
     p.out_a = static_cast<__nv_bfloat16 *>(dq);
     p.out_b = nullptr;
-    attn::bwd_dq_kernel<D><<<dim3(T / 128, BH), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
+    using Q = attn::DqCfg<D>;
+    attn::bwd_dq_kernel<D><<<dim3(T / 128, BH), Q::THREADS, Q::SMEM, stream>>>(mq, mk, mv, mg, p);
     return launch_status();
 }
 
-// Split-KV geometry of the decode path: key tiles of 128, tiles per split,
-// number of splits (every split gets at least one tile).  splits <= 0 picks
-// enough splits for about two CTAs per SM.
+// Work plan of the decode path (see decode_geometry).
 struct DecGeom {
     int nkt, nrb, balanced, chunk, eff, G, slots;
     int copies;  // copies of the packed rows in the 128-row tile (4, 2 or 1)

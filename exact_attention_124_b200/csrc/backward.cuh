@@ -417,129 +417,285 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- dQ
+// The dQ kernel keeps 128-wide score MMAs (64-wide ones run at 2/3 of the
+// rate): TMEM holds two S buffers, one dP buffer and dQ (2 x 128 + 128 + d_h
+// <= 512 columns), K and V stream through separate rings, and the MMA issue
+// order per key block n is
+//   dP(n+1) [once both warpgroups hold dP(n) in registers]
+//   dQ += dS(n) K_n [once dS(n) is written]  S(n+2) [into dS(n)'s buffer]
+// so the tensor pipe computes the next blocks' S and dP during the
+// elementwise step of block n.  Warpgroup h takes keys [64h, 64h + 64) of
+// every block and writes its dS as bf16 pairs over the first 32 of its own
+// 64 S columns.
+template <int D>
+struct DqCfg {
+    static constexpr int KB = D / 64;
+    static constexpr int SUB = 128 * 128;
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int NK = (D == 128) ? 3 : 4;   // K ring slots
+    static constexpr int NV = (D == 128) ? 2 : 3;   // V ring slots
+    static constexpr int OFF_FIX = 0;               // Q, dO
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + NK * TILE;
+    static constexpr int OFF_BAR = OFF_V + NV * TILE;
+    // fix, kfull/kempty[NK], vfull/vempty[NV], sfull[2], dpfull, dpfree, dsfull[2], done, drain
+    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 1 + 1 + 2 + 1 + 1;
+    static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    static constexpr int THREADS = 320;
+    static constexpr int MMA_WARP = 8, TMA_WARP = 9;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TM_DP = 256, TM_DQ = 384;  // S buffer b at 128 b
+    static constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false);
+    static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);
+};
+
+enum : unsigned int { W_Q_FIX = 112, W_Q_KFULL, W_Q_KEMPTY, W_Q_VFULL, W_Q_VEMPTY, W_Q_SFULL,
+                      W_Q_DPFULL, W_Q_DPFREE, W_Q_DSFULL, W_Q_DONE, W_Q_DRAIN };
+
 // grid: (T / 128 query blocks, B * H); causal: the highest query block sees
 // the most keys and starts first.
 template <int D>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+__global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const BwdParams p)
 {
-    using C = BwdCfg<D>;
+    using C = DqCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    BwdSmem<D> sm;
-    sm.init(smem_raw);
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base + C::OFF_FIX, sG = sQ + C::TILE;
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+    const uint32_t b_fix = base + C::OFF_BAR;
+    const uint32_t b_kfull = b_fix + 8, b_kempty = b_kfull + 8 * C::NK;
+    const uint32_t b_vfull = b_kempty + 8 * C::NK, b_vempty = b_vfull + 8 * C::NV;
+    const uint32_t b_sfull = b_vempty + 8 * C::NV;  // [2] S(n) in buffer n & 1
+    const uint32_t b_dpfull = b_sfull + 16;         // dP(n) computed
+    const uint32_t b_dpfree = b_dpfull + 8;         // both warpgroups hold dP(n) in registers
+    const uint32_t b_dsfull = b_dpfree + 8;         // [2] dS(n) written over buffer n & 1
+    const uint32_t b_done = b_dsfull + 16;
+    const uint32_t b_drain = b_done + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem = bwd_setup<D>(sm, warp);
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_fix, 1);
+        for (int s = 0; s < C::NK; ++s) {
+            mbar_init(b_kfull + 8 * s, 1);
+            mbar_init(b_kempty + 8 * s, 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(b_vfull + 8 * s, 1);
+            mbar_init(b_vempty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_sfull + 8 * b, 1);
+            mbar_init(b_dsfull + 8 * b, 256);
+        }
+        mbar_init(b_dpfull, 1);
+        mbar_init(b_dpfree, 256);
+        mbar_init(b_done, 1);
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
     const uint64_t lim = p.limit_ns;
     const int i = p.causal ? p.nq - 1 - (int)blockIdx.x : (int)blockIdx.x;
     const int bh = blockIdx.y;
     const int Hq = p.H_kv * p.group;
     const int kvbh = (bh / Hq) * p.H_kv + (bh % Hq) / p.group;
     const int nkb = p.causal ? i + 1 : p.nq;
-    const uint32_t sQ = sm.fix, sG = sm.fix + C::TILE;
 
     if (warp == C::TMA_WARP) {
-        if (lane == 0) {  // TMA: Q_i, dO_i once; then K_j, V_j per iteration
+        if (lane == 0) {  // TMA: Q_i, dO_i once; then K_0, V_0, K_1, V_1, K_2, ... (consumption order)
             const uint64_t pol = policy_evict_last();
-            mbar_arrive_expect_tx(sm.b_fix, 2 * C::TILE);
+            mbar_arrive_expect_tx(b_fix, 2 * C::TILE);
             for (int kb = 0; kb < C::KB; ++kb) {
-                tma_load_3d(sQ + kb * C::SUB, &tmQ, sm.b_fix, 64 * kb, 128 * i, bh, pol);
-                tma_load_3d(sG + kb * C::SUB, &tmdO, sm.b_fix, 64 * kb, 128 * i, bh, pol);
+                tma_load_3d(sQ + kb * C::SUB, &tmQ, b_fix, 64 * kb, 128 * i, bh, pol);
+                tma_load_3d(sG + kb * C::SUB, &tmdO, b_fix, 64 * kb, 128 * i, bh, pol);
             }
-            uint32_t armed = 0, armed_par = 0;
+            uint32_t karmed = 0, karmed_par = 0, varmed = 0, varmed_par = 0;
             bool ok = true;
-            for (int jj = 0; jj < nkb; ++jj) {
-                const int s = jj % C::NST;
-                const uint32_t par = (uint32_t)(jj / C::NST) & 1u;
-                if (!mbar_wait(sm.b_empty + 8 * s, par ^ 1u, lim, W_B_STEMPTY, sm.abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t st = sm.ring + s * C::STAGE;
-                mbar_arrive_expect_tx(sm.b_full + 8 * s, 2 * C::TILE);
+            auto load = [&](bool is_k, int jj) -> bool {
+                const int nsl = is_k ? C::NK : C::NV;
+                const int s = jj % nsl;
+                const uint32_t par = (uint32_t)(jj / nsl) & 1u;
+                const uint32_t full = (is_k ? b_kfull : b_vfull) + 8 * s;
+                if (!mbar_wait((is_k ? b_kempty : b_vempty) + 8 * s, par ^ 1u, lim,
+                               is_k ? W_Q_KEMPTY : W_Q_VEMPTY, abort_flag))
+                    return false;
+                mbar_arrive_expect_tx(full, C::TILE);
+                uint32_t &armed = is_k ? karmed : varmed, &apar = is_k ? karmed_par : varmed_par;
                 armed |= 1u << s;
-                armed_par = (armed_par & ~(1u << s)) | (par << s);
-                for (int kb = 0; kb < C::KB; ++kb) {
-                    tma_load_3d(st + kb * C::SUB, &tmK, sm.b_full + 8 * s, 64 * kb, 128 * jj, kvbh, pol);
-                    tma_load_3d(st + C::TILE + kb * C::SUB, &tmV, sm.b_full + 8 * s, 64 * kb,
-                                128 * jj, kvbh, pol);
-                }
+                apar = (apar & ~(1u << s)) | (par << s);
+                const uint32_t dst = (is_k ? sK : sV) + s * C::TILE;
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(dst + kb * C::SUB, is_k ? &tmK : &tmV, full, 64 * kb, 128 * jj, kvbh, pol);
+                return true;
+            };
+            // the MMA warp takes K_0, V_0, K_1, then V_n before K_{n+1} for n >= 1
+            ok = load(true, 0) && load(false, 0);
+            if (ok && nkb > 1) ok = load(true, 1);
+            for (int jj = 1; ok && jj < nkb; ++jj) {
+                ok = load(false, jj);
+                if (ok && jj + 1 < nkb) ok = load(true, jj + 1);
             }
             if (!ok) {
-                *sm.abort_flag = 1;
-                mbar_wait(sm.b_fix, 0, lim, W_B_KV);
-                for (int s = 0; s < C::NST; ++s)
-                    if ((armed >> s) & 1u) mbar_wait(sm.b_full + 8 * s, (armed_par >> s) & 1u, lim, W_B_STFULL);
+                *abort_flag = 1;
+                mbar_wait(b_fix, 0, lim, W_Q_FIX);
+                for (int s = 0; s < C::NK; ++s)
+                    if ((karmed >> s) & 1u) mbar_wait(b_kfull + 8 * s, (karmed_par >> s) & 1u, lim, W_Q_KFULL);
+                for (int s = 0; s < C::NV; ++s)
+                    if ((varmed >> s) & 1u) mbar_wait(b_vfull + 8 * s, (varmed_par >> s) & 1u, lim, W_Q_VFULL);
             }
         }
     } else if (warp == C::MMA_WARP) {
         if (lane == 0) {  // MMA issuer
-            bool ok = mbar_wait(sm.b_fix, 0, lim, W_B_KV, sm.abort_flag);
+            bool ok = mbar_wait(b_fix, 0, lim, W_Q_FIX, abort_flag);
             tc_fence_after_sync();
             const uint32_t ql = sw128_desc_lo(sQ, 16), gl = sw128_desc_lo(sG, 16);
-            auto wait_full = [&](int jj) {
-                return mbar_wait(sm.b_full + 8 * (jj % C::NST), (uint32_t)(jj / C::NST) & 1u, lim,
-                                 W_B_STFULL, sm.abort_flag);
+            auto wait_k = [&](int jj) {
+                return mbar_wait(b_kfull + 8 * (jj % C::NK), (uint32_t)(jj / C::NK) & 1u, lim, W_Q_KFULL,
+                                 abort_flag);
             };
-            auto sdp = [&](int jj, int h) {  // S = Q K_h^T, dP = dO V_h^T (64 keys)
-                const uint32_t st = sm.ring + (jj % C::NST) * C::STAGE + h * C::HALF;
-                const uint32_t kl = sw128_desc_lo(st, 16), vl = sw128_desc_lo(st + C::TILE, 16);
+            auto wait_v = [&](int jj) {
+                return mbar_wait(b_vfull + 8 * (jj % C::NV), (uint32_t)(jj / C::NV) & 1u, lim, W_Q_VFULL,
+                                 abort_flag);
+            };
+            auto s_mma = [&](int jj) {  // S(jj) = Q K_jj^T into buffer jj & 1
+                const uint32_t kl = sw128_desc_lo(sK + (jj % C::NK) * C::TILE, 16);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4;
-                    mma_ss(tmem + C::tm_s(h), sw128_desc_join(ql + off, 1024),
+                    mma_ss(tmem + 128u * (jj & 1), sw128_desc_join(ql + off, 1024),
                            sw128_desc_join(kl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
-                    mma_ss(tmem + C::tm_dp(h), sw128_desc_join(gl + off, 1024),
+                }
+                tc_commit(b_sfull + 8 * (jj & 1));
+            };
+            auto dp_mma = [&](int jj) {  // dP(jj) = dO V_jj^T
+                const int vs = jj % C::NV;
+                const uint32_t vl = sw128_desc_lo(sV + vs * C::TILE, 16);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4;
+                    mma_ss(tmem + C::TM_DP, sw128_desc_join(gl + off, 1024),
                            sw128_desc_join(vl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(sm.b_sfull + 8 * h);
+                tc_commit(b_dpfull);
+                tc_commit(b_vempty + 8 * vs);  // V_jj is free once dP(jj) has run
             };
-            auto acc = [&](int jj, int h) {  // dQ += dS_h K_h (16 keys each)
-                const uint32_t km = sw128_desc_lo(sm.ring + (jj % C::NST) * C::STAGE, C::SUB);
+            if (ok && (ok = wait_k(0))) { tc_fence_after_sync(); s_mma(0); }
+            if (ok && (ok = wait_v(0))) { tc_fence_after_sync(); dp_mma(0); }
+            if (ok && nkb > 1 && (ok = wait_k(1))) { tc_fence_after_sync(); s_mma(1); }
+            for (int n = 0; ok && n < nkb; ++n) {
+                if (n + 1 < nkb) {  // dP(n+1) once dP(n) is out of TMEM
+                    if (!(ok = mbar_wait(b_dpfree, (uint32_t)n & 1u, lim, W_Q_DPFREE, abort_flag))) break;
+                    if (!(ok = wait_v(n + 1))) break;
+                    tc_fence_after_sync();
+                    dp_mma(n + 1);
+                }
+                if (!(ok = mbar_wait(b_dsfull + 8 * (n & 1), (uint32_t)(n >> 1) & 1u, lim, W_Q_DSFULL,
+                                     abort_flag)))
+                    break;
+                tc_fence_after_sync();
+                // dQ += dS(n) K_n: keys [64h, 64h + 64) sit at columns 64h + [0, 32) as bf16 pairs
+                const uint32_t km = sw128_desc_lo(sK + (n % C::NK) * C::TILE, C::SUB);
+                const uint32_t tds = tmem + 128u * (n & 1);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + C::TM_ACC0, tmem + C::tm_s(h) + 8 * kk,
-                           sw128_desc_join(km + (uint32_t)(4 * h + kk) * (2048 >> 4), 1024),
-                           C::IDESC_ACC, (jj > 0 || h > 0 || kk > 0) ? 1u : 0u);
-            };
-            ok = ok && bwd_mma_loop(nkb, sm.b_pfull, sm.b_empty, lim, sm.abort_flag, sdp, acc,
-                                    wait_full, C::NST);
-            if (!ok) *sm.abort_flag = 1;
-            tc_commit(sm.b_done);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::TM_DQ, tds + 64 * (kk >> 2) + 8 * (kk & 3),
+                           sw128_desc_join(km + kk * (2048 >> 4), 1024), C::IDESC_ACC,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(b_kempty + 8 * (n % C::NK));  // K_n's last use
+                if (n + 2 < nkb) {  // S(n+2) into the buffer dQ just read (in issue order)
+                    if (!(ok = wait_k(n + 2))) break;
+                    tc_fence_after_sync();
+                    s_mma(n + 2);
+                }
+            }
+            if (!ok) *abort_flag = 1;
+            tc_commit(b_done);  // fires when every MMA issued above has completed
         }
-    } else if (warp < 8) {  // elementwise warpgroup h: thread = query row, keys of half h
+    } else if (warp < 8) {  // elementwise warpgroup h: thread = query row, keys [64h, 64h + 64)
         const int h = warp >> 2;
         const int qr = (warp & 3) * 32 + lane;
         const int row = 128 * i + qr;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const float2 st_row = p.stats[(size_t)bh * p.T + row];
+        const float2 st = p.stats[(size_t)bh * p.T + row];
+        const float cl2 = p.c_log2;
         bool ok = true;
-        for (int jj = 0; ok && jj < nkb; ++jj) {
-            const bool w = mbar_wait(sm.b_sfull + 8 * h, (uint32_t)jj & 1u, lim, W_B_SFULL, sm.abort_flag);
+        for (int n = 0; ok && n < nkb; ++n) {
+            bool w = mbar_wait(b_sfull + 8 * (n & 1), (uint32_t)(n >> 1) & 1u, lim, W_Q_SFULL, abort_flag);
+            w = w && mbar_wait(b_dpfull, (uint32_t)n & 1u, lim, W_Q_DPFULL, abort_flag);
             if (!(ok = __all_sync(0xffffffffu, w))) break;
             tc_fence_after_sync();
-            const bool need_mask = p.causal && jj == i;
-            bwd_elementwise<false, false>(tmem + lane_off + C::tm_s(h), tmem + lane_off + C::tm_dp(h),
-                                          p.c_log2, nullptr, st_row, need_mask, row,
-                                          128 * jj + 64 * h, tmem + lane_off + C::tm_s(h),
-                                          sm.b_pfull + 8 * h);
+            const uint32_t tS = tmem + lane_off + 128u * (n & 1) + 64 * h;
+            const uint32_t tD = tmem + lane_off + C::TM_DP + 64 * h;
+            uint32_t rs[64], rd[64];
+            {
+                uint32_t a[32], b2[32], c[32], d[32];
+                tmem_ld32(tS, a);
+                tmem_ld32(tS + 32, b2);
+                tmem_ld32(tD, c);
+                tmem_ld32(tD + 32, d);
+                tmem_wait_ld_regs(a);
+                tmem_wait_ld_regs(b2);
+                tmem_wait_ld_regs(c);
+                tmem_wait_ld_regs(d);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    rs[x] = a[x];
+                    rs[32 + x] = b2[x];
+                    rd[x] = c[x];
+                    rd[32 + x] = d[x];
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(b_dpfree);  // dP(n) is in registers: dP(n+1) may overwrite it
+            const bool need_mask = p.causal && n == i;
+            const int key0 = 128 * n + 64 * h;
+            uint32_t dk[32];
+#pragma unroll
+            for (int q = 0; q < 64; q += 2) {
+                float dsr[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float pv = fast_exp2(fmaf(__uint_as_float(rs[q + e]), cl2, -st.x));
+                    if (need_mask && key0 + q + e > row) pv = 0.f;
+                    dsr[e] = pv * (__uint_as_float(rd[q + e]) - st.y);
+                }
+                dk[q >> 1] = pack_bf16x2(dsr[0], dsr[1]);
+            }
+            tmem_st32(tS, dk);
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(b_dsfull + 8 * (n & 1));
         }
-        const bool w = ok && mbar_wait(sm.b_done, 0, lim, W_B_DONE, sm.abort_flag);
-        if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
+        const bool w = ok && mbar_wait(b_done, 0, lim, W_Q_DONE, abort_flag);
+        if (__all_sync(0xffffffffu, w) && !*abort_flag) {
             tc_fence_after_sync();
             __nv_bfloat16 *dst = p.out_a + ((size_t)bh * p.T + row) * D;
             if (h == 0)  // the two warpgroups store the two halves of the d_h columns
-                store_rows<0, D / 64>(tmem + lane_off + C::TM_ACC0, p.scale, dst);
+                store_rows<0, D / 64>(tmem + lane_off + C::TM_DQ, p.scale, dst);
             else
-                store_rows<D / 64, D / 32>(tmem + lane_off + C::TM_ACC0, p.scale, dst);
+                store_rows<D / 64, D / 32>(tmem + lane_off + C::TM_DQ, p.scale, dst);
         } else {
-            *sm.abort_flag = 1;
+            *abort_flag = 1;
         }
     }
-    if (warp == C::MMA_WARP && lane == 0 && *sm.abort_flag) {
-        tc_commit(sm.b_drain);
-        mbar_wait(sm.b_drain, 0, lim, W_B_DRAIN);
+    if (warp == C::MMA_WARP && lane == 0 && *abort_flag) {
+        tc_commit(b_drain);
+        mbar_wait(b_drain, 0, lim, W_Q_DRAIN);
     }
     tc_fence_before_sync();
     __syncthreads();
