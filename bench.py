@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--exp-split", type=int, default=None,
                     help="fused kernel variant: column pairs of every 8 whose exponentials run "
                          "on the FMA pipe (0, 2, 3, 4); default: the library's choice")
+    ap.add_argument("--key-tile", type=int, default=None, choices=[64, 128],
+                    help="fused kernel variant: key tile 64 (two score buffers per query tile) "
+                         "or 128; default: the library's choice")
     args = ap.parse_args()
     if args.e2e_steps < 1 or args.steps < 1:
         ap.error("--steps and --e2e-steps must be at least 1")
@@ -299,6 +302,8 @@ def run_ours(args):
     attn.load_library()
     if args.exp_split is not None:
         attn.set_exp_split(args.exp_split)
+    if args.key_tile is not None:
+        attn.set_key_tile(args.key_tile)
     peaks, peak_src = load_peaks()
     if args.path == "unfused":
         return run_unfused(args, w, world, rank, local, peaks, peak_src)

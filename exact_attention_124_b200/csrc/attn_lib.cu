@@ -13,6 +13,7 @@
 #include "attn.h"
 #include "attn_selftest.h"
 #include "backward.cuh"
+#include "fused_fwd_k64.cuh"
 #include "decode.cuh"
 #include "fused_fwd.cuh"
 #include "selftest.cuh"
@@ -26,6 +27,8 @@ constexpr int kMaxDevices = 64;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_mma_order = 0;
 int g_exp_split = -1;  // pairs of every 8 on the FMA pipe; -1: per-head-size default
+int g_key_tile = 0;    // fused forward key tile: 64 or 128; 0: per-head-size default
+constexpr int kDefaultKeyTile64 = 128, kDefaultKeyTile128 = 128;
 constexpr int kDefaultSplit64 = 0, kDefaultSplit128 = 0;  // measured fastest on B200
 unsigned int g_last_where = 0;
 
@@ -104,10 +107,20 @@ bool fused_ready()
 }
 
 template <int D>
+bool fused_k64_ready()
+{
+    using C = attn::FusedK64Cfg<D>;
+    if (!set_smem(attn::attn_fwd_fused_k64_kernel<D>, C::SMEM)) return false;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn::attn_fwd_fused_k64_kernel<D>) != cudaSuccess) return false;
+    return fa.numRegs >= C::REGS_LAUNCH && fa.maxThreadsPerBlock >= C::THREADS;
+}
+
+template <int D>
 bool fused_all_ready()
 {
     return fused_ready<D, 0>() && fused_ready<D, 2>() && fused_ready<D, 3>() &&
-           fused_ready<D, 4>();
+           fused_ready<D, 4>() && fused_k64_ready<D>();
 }
 
 // Per-device one-time set-up: device check (compute capability 10.0),
@@ -236,6 +249,15 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     p.order_mode = g_mma_order;
     p.limit_ns = kWaitLimitNs;
     const int grid = fused_grid(BH, T, causal, sms);
+    const int key_tile = g_key_tile > 0 ? g_key_tile : (D == 64 ? kDefaultKeyTile64 : kDefaultKeyTile128);
+    if (key_tile == 64) {  // 64-key tiles, two score buffers per query tile (all exps on MUFU)
+        using C64 = attn::FusedK64Cfg<D>;
+        if (make_map(&mk, k, D, T, (uint64_t)B * H_kv, 64) ||
+            make_map(&mv, v, D, T, (uint64_t)B * H_kv, 64))
+            return ATTN_ERR_LAUNCH;
+        attn::attn_fwd_fused_k64_kernel<D><<<grid, C64::THREADS, C64::SMEM, stream>>>(mq, mk, mv, p);
+        return launch_status();
+    }
     const int split = g_exp_split >= 0 ? g_exp_split : (D == 64 ? kDefaultSplit64 : kDefaultSplit128);
     switch (split) {
         case 0: attn::attn_fwd_fused_kernel<D, 0><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
@@ -709,6 +731,14 @@ int attn_selftest_set_mma_order(int mode)
 }
 
 int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
+
+int attn_selftest_set_key_tile(int keys)
+{
+    if (keys != 0 && keys != 64 && keys != 128) return -1;
+    const int prev = g_key_tile;
+    g_key_tile = keys;
+    return prev;
+}
 
 int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms,
                               int *segs, int seg_cap, int *nseg, int nseg_cap, int *slots,

@@ -72,6 +72,16 @@ int attn_selftest_set_exp_split(int pairs_of_8);
 int attn_selftest_last_wait_site(void);
 
 /*
+ * Key tile of the fused forward: 128 (P written over the score tile; the
+ * exp-split variants apply) or 64 (two score buffers per query tile, the next
+ * score MMA overlapping the softmax; all exponentials on MUFU); 0 restores
+ * the per-head-size default.  Same arithmetic up to the order of the online
+ * softmax's rescaling.  Returns the previous setting (0 = default), or -1 for
+ * another value.
+ */
+int attn_selftest_set_key_tile(int keys);
+
+/*
  * Host only (no device needed): the work plan attn_fwd_decode would launch
  * for these sizes and `splits` on a device with `sms` SMs, computed by the
  * same code the kernel runs.  A head is (batch * H_kv + K/V head, block of 128
