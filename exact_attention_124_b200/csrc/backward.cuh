@@ -15,17 +15,17 @@
 //                     dV += P^T dO and dK += dS^T Q accumulate in TMEM
 //   bwd_dq_kernel     one CTA per (query head, 128 queries): loops over the key
 //                     blocks it sees; S and dP into TMEM, dS back as bf16,
-//                     dQ += dS K in TMEM
-// Each 128-wide block of the moving operand is taken as two 64-wide halves,
-// half h in TMEM buffer h and handled by elementwise warpgroup h, so the
-// tensor cores compute one half's S/dP and accumulate the other's gradient
-// while a warpgroup does the elementwise step (a two-buffer ping-pong; TMEM
-// has room for two 64-column S/dP pairs next to the 2 d_h accumulator
-// columns, not for two 128-column ones).
-// Warps: 0-3 / 4-7 elementwise warpgroups 0 / 1 (thread = TMEM lane = the
-// stationary block's row), warp 8 issues MMAs, warp 9 issues TMA copies.
-// TMEM: buffer h = S/P [128h, 128h + 64), dP/dS [128h + 64, 128h + 128);
-// accumulators from 256.
+//                     dQ += dS K in TMEM (its own schedule: see DqCfg below)
+// Both gradient kernels: warps 0-3 / 4-7 are elementwise warpgroups 0 / 1
+// (thread = TMEM lane = the stationary block's row), warp 8 issues MMAs,
+// warp 9 issues TMA copies.
+// dK/dV kernel: each 128-wide block of queries is taken as two 64-wide
+// halves, half h in TMEM buffer h and handled by elementwise warpgroup h, so
+// the tensor cores compute one half's S/dP and accumulate the other's
+// gradient while a warpgroup does the elementwise step (a two-buffer
+// ping-pong; TMEM has room for two 64-column S/dP pairs next to the 2 d_h
+// accumulator columns, not for two 128-column ones).  TMEM: buffer h = S/P
+// [128h, 128h + 64), dP/dS [128h + 64, 128h + 128); accumulators from 256.
 #pragma once
 
 #include "sm100.cuh"
