@@ -305,12 +305,12 @@ def run_ours(args):
     if args.key_tile is not None:
         attn.set_key_tile(args.key_tile)
     peaks, peak_src = load_peaks()
-    if args.path == "unfused":
-        return run_unfused(args, w, world, rank, local, peaks, peak_src)
-    if args.path == "backward":
-        return run_backward(args, w, world, rank, local, peaks, peak_src)
-    if args.path == "decode":
-        return run_decode(args, w, world, rank, local, peaks, peak_src)
+    other = {"unfused": run_unfused, "backward": run_backward, "decode": run_decode}.get(args.path)
+    if other is not None:
+        rc = other(args, w, world, rank, local, peaks, peak_src)
+        if world > 1:
+            dist.destroy_process_group()
+        return rc
 
     # inputs: per-rank seed, generated on the host, copied once (resident in HBM)
     q, k, v = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)
