@@ -64,11 +64,13 @@ def load_library():
     lib.attn_selftest_set_exp_split.argtypes = [I]
     lib.attn_selftest_decode_plan.argtypes = [I, I, I, I, I, I, I, P, I, P, I, P, P]
     lib.attn_selftest_set_key_tile.argtypes = [I]
+    lib.attn_selftest_fused_plan.argtypes = [I, I, I, I, I, I, P, I, P]
     for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_decode", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
                  "attn_selftest_last_wait_site", "attn_selftest_set_exp_split",
-                 "attn_selftest_decode_plan", "attn_selftest_set_key_tile"):
+                 "attn_selftest_decode_plan", "attn_selftest_set_key_tile",
+                 "attn_selftest_fused_plan"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -265,6 +267,23 @@ def set_exp_split(pairs_of_8: int) -> int:
     if prev == -2:
         raise ValueError("exp split must be -1, 0, 2, 3 or 4")
     return prev
+
+
+def fused_plan(B: int, H: int, H_kv: int, T: int, causal: bool, sms: int):
+    """Host-side work units of the fused forward on a device with ``sms`` SMs
+    (no device needed): (units, ctas) with units a list of
+    (cta, k, query_head, kv_head, first_row, n0, n1) tuples."""
+    lib = load_library()
+    ctas = ctypes.c_int(0)
+    n = lib.attn_selftest_fused_plan(B, H, H_kv, T, int(bool(causal)), sms, None, 0,
+                                     ctypes.byref(ctas))
+    if n < 0:
+        raise ValueError("bad sizes")
+    buf = (ctypes.c_int * (7 * max(n, 1)))()
+    n2 = lib.attn_selftest_fused_plan(B, H, H_kv, T, int(bool(causal)), sms, buf, n,
+                                      ctypes.byref(ctas))
+    assert n2 == n
+    return [tuple(buf[7 * i:7 * i + 7]) for i in range(n)], ctas.value
 
 
 def decode_plan(B: int, H: int, H_kv: int, Tq: int, Tk: int, splits: int, sms: int):

@@ -224,6 +224,26 @@ int fused_grid(long long BH, int T, int causal, int sms)
     return (int)(work < sms ? work : sms);
 }
 
+// Kernel parameters of a fused launch (output pointers left null).
+attn::FusedParams fused_params(int B, int H, int H_kv, int T, int causal, float scale)
+{
+    attn::FusedParams p;
+    p.o = nullptr;
+    p.lse = nullptr;
+    p.BH = B * H;
+    p.H = H;
+    p.group = H / H_kv;
+    p.T = T;
+    p.causal = causal;
+    p.c_log2 = scale * 1.4426950408889634f;
+    p.nqb = (T + 255) / 256;
+    p.units = p.BH * p.nqb;
+    p.nkv = (T + 127) / 128;
+    p.order_mode = g_mma_order;
+    p.limit_ns = kWaitLimitNs;
+    return p;
+}
+
 template <int D>
 int launch_fused(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
                  int H_kv, int T, int causal, float scale, cudaStream_t stream, int sms)
@@ -234,20 +254,9 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, (uint64_t)B * H_kv, 128) ||
         make_map(&mv, v, D, T, (uint64_t)B * H_kv, 128))
         return ATTN_ERR_LAUNCH;
-    attn::FusedParams p;
+    attn::FusedParams p = fused_params(B, H, H_kv, T, causal, scale);
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
-    p.BH = BH;
-    p.H = H;
-    p.group = H / H_kv;
-    p.T = T;
-    p.causal = causal;
-    p.c_log2 = scale * 1.4426950408889634f;
-    p.nqb = (T + 255) / 256;
-    p.units = BH * p.nqb;
-    p.nkv = (T + 127) / 128;
-    p.order_mode = g_mma_order;
-    p.limit_ns = kWaitLimitNs;
     const int grid = fused_grid(BH, T, causal, sms);
     const int key_tile = g_key_tile > 0 ? g_key_tile : (D == 64 ? kDefaultKeyTile64 : kDefaultKeyTile128);
     if (key_tile == 64) {  // 64-key tiles, two score buffers per query tile (all exps on MUFU)
@@ -738,6 +747,32 @@ int attn_selftest_set_key_tile(int keys)
     const int prev = g_key_tile;
     g_key_tile = keys;
     return prev;
+}
+
+int attn_selftest_fused_plan(int B, int H, int H_kv, int T, int causal, int sms, int *units,
+                             int cap, int *ctas)
+{
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || T < 1 || sms < 1 ||
+        (causal != 0 && causal != 1) || (long long)B * H * (long long)T > (long long)INT_MAX)
+        return -1;
+    const attn::FusedParams p = fused_params(B, H, H_kv, T, causal, 1.f);
+    const int G = fused_grid((long long)B * H, T, causal, sms);
+    if (ctas) *ctas = G;
+    long long nrec = 0;
+    for (int c = 0; c < G; ++c) {
+        attn::UnitInfo u;
+        for (int k = 0;; ++k) {
+            const int r = attn::unit_of_cta(p, G, c, k, u);
+            if (r < 0) break;
+            if (r == 0) continue;
+            if (units && nrec < cap) {
+                int *x = units + 7 * nrec;
+                x[0] = c; x[1] = k; x[2] = u.bh; x[3] = u.kvh; x[4] = u.i0; x[5] = u.n[0]; x[6] = u.n[1];
+            }
+            ++nrec;
+        }
+    }
+    return nrec > INT_MAX ? INT_MAX : (int)nrec;
 }
 
 int attn_selftest_decode_plan(int B, int H, int H_kv, int Tq, int Tk, int splits, int sms,

@@ -182,15 +182,15 @@ struct UnitInfo {
 };
 
 // Pairs per head in causal mode (query block q with nqb-1-q).
-__device__ __forceinline__ int pairs_per_head(const FusedParams &p) { return (p.nqb + 1) >> 1; }
+__host__ __device__ __forceinline__ int pairs_per_head(const FusedParams &p) { return (p.nqb + 1) >> 1; }
 
-// The k-th unit of this CTA.  Returns 1 with `u` filled, 0 for a hole (the
-// middle block of an odd nqb appears once per pair list), -1 when the CTA has
-// no more work.  Every role of the CTA walks the same sequence.
-__device__ __forceinline__ int unit_of(const FusedParams &p, int k, UnitInfo &u)
+// The k-th unit of CTA c of a grid of G CTAs.  Returns 1 with `u` filled, 0
+// for a hole (the middle block of an odd nqb appears once per pair list), -1
+// when the CTA has no more work.  Every role of the CTA walks the same
+// sequence.  Also run on the host by attn_selftest_fused_plan().
+__host__ __device__ __forceinline__ int unit_of_cta(const FusedParams &p, int G, int c, int k,
+                                                    UnitInfo &u)
 {
-    const int G = (int)gridDim.x;
-    const int c = (int)blockIdx.x;
     int qb;
     if (p.causal) {
         const int npp = pairs_per_head(p);
@@ -223,6 +223,11 @@ __device__ __forceinline__ int unit_of(const FusedParams &p, int k, UnitInfo &u)
     }
     u.niter = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
     return 1;
+}
+
+__device__ __forceinline__ int unit_of(const FusedParams &p, int k, UnitInfo &u)
+{
+    return unit_of_cta(p, (int)gridDim.x, (int)blockIdx.x, k, u);
 }
 
 struct Ring {

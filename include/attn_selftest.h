@@ -82,6 +82,20 @@ int attn_selftest_last_wait_site(void);
 int attn_selftest_set_key_tile(int keys);
 
 /*
+ * Host only (no device needed): the work units the fused forward would run
+ * for these sizes on a device with `sms` SMs, computed by the kernel's own
+ * unit function.  A unit is 256 query rows of one query head: two 128-row
+ * tiles that see n0 and n1 key tiles of 128.
+ *   units : up to `cap` records of 7 ints (cta, k-th unit of that CTA, query
+ *           head b * H + h, K/V head, first query row, n0, n1)
+ *   ctas  : the grid the launch would use
+ * Returns the number of units (records beyond `cap` are not written), or -1
+ * for bad sizes.
+ */
+int attn_selftest_fused_plan(int B, int H, int H_kv, int T, int causal, int sms, int *units,
+                             int cap, int *ctas);
+
+/*
  * Host only (no device needed): the work plan attn_fwd_decode would launch
  * for these sizes and `splits` on a device with `sms` SMs, computed by the
  * same code the kernel runs.  A head is (batch * H_kv + K/V head, block of 128
