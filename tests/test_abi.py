@@ -42,6 +42,30 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(raw, name), name
 
 
+def declared_parameter_counts():
+    """Parameter count of every declared function, from the headers."""
+    counts = {}
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"\b(attn_\w+)\s*\(([^)]*)\)\s*;", text):
+            params = m.group(2).strip()
+            counts[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return counts
+
+
+def test_binding_signatures_match_the_headers(lib):
+    """Every ctypes signature the binding sets has the headers' parameter count."""
+    counts = declared_parameter_counts()
+    assert set(counts) == set(declared_functions())
+    checked = 0
+    for name, n in counts.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is not None:
+            assert len(argtypes) == n, (name, len(argtypes), n)
+            checked += 1
+    assert checked >= 15
+
+
 NULL = None
 A = 4096  # a 16-byte aligned fake address: never dereferenced, validation fails first
 
