@@ -145,6 +145,7 @@ int device_ready(int *sms_out)
         if (get_encoder() != ATTN_OK) return ATTN_ERR_LAUNCH;
         bool ok = true;
         ok &= set_smem(attn::bwd_dkdv_kernel<64>, attn::BwdCfg<64>::SMEM);
+        ok &= set_smem(attn::bwd_dkdv64_kernel, attn::Dkdv64Cfg::SMEM);
         ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<64>, attn::DqCfg<64>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<128>, attn::DqCfg<128>::SMEM);
@@ -334,7 +335,11 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.limit_ns = kWaitLimitNs;
     p.out_a = static_cast<__nv_bfloat16 *>(dk);
     p.out_b = static_cast<__nv_bfloat16 *>(dv);
-    attn::bwd_dkdv_kernel<D><<<dim3(T / 128, BHkv), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
+    if (D == 64)  // room for 128-wide score MMAs and two S^T buffers at d_h = 64
+        attn::bwd_dkdv64_kernel<<<dim3(T / 128, BHkv), attn::Dkdv64Cfg::THREADS, attn::Dkdv64Cfg::SMEM,
+                                  stream>>>(mq, mk, mv, mg, p);
+    else
+        attn::bwd_dkdv_kernel<D><<<dim3(T / 128, BHkv), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
     if (launch_status()) return ATTN_ERR_LAUNCH;
     p.out_a = static_cast<__nv_bfloat16 *>(dq);
     p.out_b = nullptr;

@@ -19,7 +19,9 @@
 // Both gradient kernels: warps 0-3 / 4-7 are elementwise warpgroups 0 / 1
 // (thread = TMEM lane = the stationary block's row), warp 8 issues MMAs,
 // warp 9 issues TMA copies.
-// dK/dV kernel: each 128-wide block of queries is taken as two 64-wide
+// At d_h = 64 the dK/dV pass runs bwd_dkdv64_kernel (the dQ kernel's
+// schedule: 128-wide score MMAs, two S^T buffers).  dK/dV kernel at d_h =
+// 128: each 128-wide block of queries is taken as two 64-wide
 // halves, half h in TMEM buffer h and handled by elementwise warpgroup h, so
 // the tensor cores compute one half's S/dP and accumulate the other's
 // gradient while a warpgroup does the elementwise step (a two-buffer
@@ -409,6 +411,283 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (warp == C::MMA_WARP && lane == 0 && *sm.abort_flag) {
         tc_commit(sm.b_drain);
         mbar_wait(sm.b_drain, 0, lim, W_B_DRAIN);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- dK, dV at d_h = 64
+// At d_h = 64 the two accumulators take 128 TMEM columns, which leaves room
+// for the dQ kernel's schedule with 128-wide score MMAs: two S^T buffers, one
+// dP^T buffer, and per query block n
+//   dP^T(n+1) [once both warpgroups hold dP^T(n) in registers]
+//   dV += P^T(n) dO_n, dK += dS^T(n) Q_n [once P^T, dS^T are written]
+//   S^T(n+2) [into the buffer just read]
+// Warpgroup h takes queries [64h, 64h + 64) of every block and writes its
+// P^T and dS^T as bf16 pairs over its own 64 S^T columns (P^T first 32,
+// dS^T last 32).  TMEM: S^T buffer b [128b, 128b + 128), dP^T [256, 384),
+// dV [384, 448), dK [448, 512).
+struct Dkdv64Cfg {
+    static constexpr int D = 64;
+    static constexpr int TILE = 128 * D * 2;        // 16 KB
+    static constexpr int NST = 5;                   // stages: Q, dO and statistics of a block
+    static constexpr int STAGE = 2 * TILE + 1024;
+    static constexpr int OFF_FIX = 0;               // K, V
+    static constexpr int OFF_RING = 2 * TILE;
+    static constexpr int OFF_BAR = OFF_RING + NST * STAGE;
+    // fix, full/empty[NST], sfull[2], dpfull, dpfree, pfull[2], done, drain
+    static constexpr int NBAR = 1 + 2 * NST + 2 + 1 + 1 + 2 + 1 + 1;
+    static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    static constexpr int THREADS = 320;
+    static constexpr int MMA_WARP = 8, TMA_WARP = 9;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TM_DP = 256, TM_DV = 384, TM_DK = 448;  // S^T buffer b at 128 b
+    static constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false);
+    static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);
+};
+
+// grid: (T / 128 key blocks, B * H_kv), as bwd_dkdv_kernel.
+__global__ void __launch_bounds__(Dkdv64Cfg::THREADS, 1)
+    bwd_dkdv64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                      const BwdParams p)
+{
+    using C = Dkdv64Cfg;
+    constexpr int D = C::D;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sK = base + C::OFF_FIX, sV = sK + C::TILE, ring = base + C::OFF_RING;
+    const uint32_t b_fix = base + C::OFF_BAR;
+    const uint32_t b_full = b_fix + 8, b_empty = b_full + 8 * C::NST;
+    const uint32_t b_sfull = b_empty + 8 * C::NST;  // [2] S^T(n) in buffer n & 1
+    const uint32_t b_dpfull = b_sfull + 16;         // dP^T(n) computed
+    const uint32_t b_dpfree = b_dpfull + 8;         // both warpgroups hold dP^T(n) in registers
+    const uint32_t b_pfull = b_dpfree + 8;          // [2] P^T(n), dS^T(n) written over buffer n & 1
+    const uint32_t b_done = b_pfull + 16;
+    const uint32_t b_drain = b_done + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_fix, 1);
+        for (int s2 = 0; s2 < C::NST; ++s2) {
+            mbar_init(b_full + 8 * s2, 1);
+            mbar_init(b_empty + 8 * s2, 1);
+        }
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(b_sfull + 8 * b2, 1);
+            mbar_init(b_pfull + 8 * b2, 256);
+        }
+        mbar_init(b_dpfull, 1);
+        mbar_init(b_dpfree, 256);
+        mbar_init(b_done, 1);
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t lim = p.limit_ns;
+    const int j = blockIdx.x;
+    const int kvbh = blockIdx.y;
+    const int b = kvbh / p.H_kv, kvl = kvbh % p.H_kv;
+    const int i0 = p.causal ? j : 0;
+    const int per_head = p.nq - i0;
+    const int niter = p.group * per_head;
+
+    if (warp == C::TMA_WARP) {
+        if (lane == 0) {  // TMA: K_j, V_j once; then Q_i, dO_i, statistics per query block
+            const uint64_t pol = policy_evict_last();
+            mbar_arrive_expect_tx(b_fix, 2 * C::TILE);
+            tma_load_3d(sK, &tmK, b_fix, 0, 128 * j, kvbh, pol);
+            tma_load_3d(sV, &tmV, b_fix, 0, 128 * j, kvbh, pol);
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int n = 0; n < niter; ++n) {
+                const int s2 = n % C::NST;
+                const uint32_t par = (uint32_t)(n / C::NST) & 1u;
+                if (!mbar_wait(b_empty + 8 * s2, par ^ 1u, lim, W_B_STEMPTY, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int g = n / per_head, i = i0 + n % per_head;
+                const int bh = b * (p.H_kv * p.group) + kvl * p.group + g;
+                const uint32_t st = ring + s2 * C::STAGE;
+                mbar_arrive_expect_tx(b_full + 8 * s2, 2 * C::TILE + 1024);
+                armed |= 1u << s2;
+                armed_par = (armed_par & ~(1u << s2)) | (par << s2);
+                tma_load_3d(st, &tmQ, b_full + 8 * s2, 0, 128 * i, bh, pol);
+                tma_load_3d(st + C::TILE, &tmdO, b_full + 8 * s2, 0, 128 * i, bh, pol);
+                bulk_load(st + 2 * C::TILE, p.stats + (size_t)bh * p.T + 128 * i, 1024, b_full + 8 * s2);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                mbar_wait(b_fix, 0, lim, W_B_KV);
+                for (int s2 = 0; s2 < C::NST; ++s2)
+                    if ((armed >> s2) & 1u) mbar_wait(b_full + 8 * s2, (armed_par >> s2) & 1u, lim, W_B_STFULL);
+            }
+        }
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {  // MMA issuer
+            bool ok = mbar_wait(b_fix, 0, lim, W_B_KV, abort_flag);
+            tc_fence_after_sync();
+            const uint32_t kl = sw128_desc_lo(sK, 16), vl = sw128_desc_lo(sV, 16);
+            auto stage = [&](int n) { return ring + (n % C::NST) * C::STAGE; };
+            auto wait_full = [&](int n) {
+                return mbar_wait(b_full + 8 * (n % C::NST), (uint32_t)(n / C::NST) & 1u, lim, W_B_STFULL,
+                                 abort_flag);
+            };
+            auto s_mma = [&](int n) {  // S^T(n) = K Q_n^T into buffer n & 1
+                const uint32_t ql = sw128_desc_lo(stage(n), 16);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(kk * 32) >> 4;
+                    mma_ss(tmem + 128u * (n & 1), sw128_desc_join(kl + off, 1024),
+                           sw128_desc_join(ql + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(b_sfull + 8 * (n & 1));
+            };
+            auto dp_mma = [&](int n) {  // dP^T(n) = V dO_n^T
+                const uint32_t gl = sw128_desc_lo(stage(n) + C::TILE, 16);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(kk * 32) >> 4;
+                    mma_ss(tmem + C::TM_DP, sw128_desc_join(vl + off, 1024),
+                           sw128_desc_join(gl + off, 1024), C::IDESC_SQ, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(b_dpfull);
+            };
+            if (ok && (ok = wait_full(0))) {
+                tc_fence_after_sync();
+                s_mma(0);
+                dp_mma(0);
+            }
+            if (ok && niter > 1 && (ok = wait_full(1))) {
+                tc_fence_after_sync();
+                s_mma(1);
+            }
+            for (int n = 0; ok && n < niter; ++n) {
+                if (n + 1 < niter) {  // dP^T(n+1) once dP^T(n) is out of TMEM (stage n+1 is in)
+                    if (!(ok = mbar_wait(b_dpfree, (uint32_t)n & 1u, lim, W_B_PFULL, abort_flag))) break;
+                    tc_fence_after_sync();
+                    dp_mma(n + 1);
+                }
+                if (!(ok = mbar_wait(b_pfull + 8 * (n & 1), (uint32_t)(n >> 1) & 1u, lim, W_B_PFULL,
+                                     abort_flag)))
+                    break;
+                tc_fence_after_sync();
+                // dV += P^T dO_n, dK += dS^T Q_n: queries [64h, 64h + 64) at columns 64h + [0, 32)
+                // (P^T) and 64h + [32, 64) (dS^T) as bf16 pairs
+                const uint32_t st = stage(n);
+                const uint32_t qm = sw128_desc_lo(st, 16384), gm = sw128_desc_lo(st + C::TILE, 16384);
+                const uint32_t tb = tmem + 128u * (n & 1);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = (n > 0 || kk > 0) ? 1u : 0u;
+                    const uint32_t col = 64u * (kk >> 2) + 8u * (kk & 3);
+                    const uint32_t boff = (uint32_t)kk * (2048 >> 4);
+                    mma_ts(tmem + C::TM_DV, tb + col, sw128_desc_join(gm + boff, 1024), C::IDESC_ACC, a);
+                    mma_ts(tmem + C::TM_DK, tb + col + 32, sw128_desc_join(qm + boff, 1024), C::IDESC_ACC, a);
+                }
+                tc_commit(b_empty + 8 * (n % C::NST));  // Q_n, dO_n and the statistics are used up
+                if (n + 2 < niter) {  // S^T(n+2) into the buffer just read (in issue order)
+                    if (!(ok = wait_full(n + 2))) break;
+                    tc_fence_after_sync();
+                    s_mma(n + 2);
+                }
+            }
+            if (!ok) *abort_flag = 1;
+            tc_commit(b_done);
+        }
+    } else if (warp < 8) {  // elementwise warpgroup h: thread = key row, queries [64h, 64h + 64)
+        const int h = warp >> 2;
+        const int kr = (warp & 3) * 32 + lane;
+        const int key = 128 * j + kr;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const float cl2 = p.c_log2;
+        bool ok = true;
+        for (int n = 0; ok && n < niter; ++n) {
+            const int s2 = n % C::NST;
+            const int i = i0 + n % per_head;
+            bool w = mbar_wait(b_full + 8 * s2, (uint32_t)(n / C::NST) & 1u, lim, W_B_STFULL, abort_flag);
+            w = w && mbar_wait(b_sfull + 8 * (n & 1), (uint32_t)(n >> 1) & 1u, lim, W_B_SFULL, abort_flag);
+            w = w && mbar_wait(b_dpfull, (uint32_t)n & 1u, lim, W_B_SFULL, abort_flag);
+            if (!(ok = __all_sync(0xffffffffu, w))) break;
+            tc_fence_after_sync();
+            const uint32_t tS = tmem + lane_off + 128u * (n & 1) + 64 * h;
+            const uint32_t tD = tmem + lane_off + C::TM_DP + 64 * h;
+            uint32_t rs[64], rd[64];
+            {
+                uint32_t a0[32], a1[32], d0[32], d1[32];
+                tmem_ld32(tS, a0);
+                tmem_ld32(tS + 32, a1);
+                tmem_ld32(tD, d0);
+                tmem_ld32(tD + 32, d1);
+                tmem_wait_ld_regs(a0);
+                tmem_wait_ld_regs(a1);
+                tmem_wait_ld_regs(d0);
+                tmem_wait_ld_regs(d1);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    rs[x] = a0[x];
+                    rs[32 + x] = a1[x];
+                    rd[x] = d0[x];
+                    rd[32 + x] = d1[x];
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(b_dpfree);  // dP^T(n) is in registers: dP^T(n+1) may overwrite it
+            const float2 *stc =
+                reinterpret_cast<const float2 *>(gbase + C::OFF_RING + s2 * C::STAGE + 2 * C::TILE) + 64 * h;
+            const bool need_mask = p.causal && i == j;
+            const int q0 = 128 * i + 64 * h;
+            uint32_t pk[32], dk[32];
+#pragma unroll
+            for (int q = 0; q < 64; q += 2) {
+                float pr[2], dsr[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float2 sd = stc[q + e];
+                    float pv = fast_exp2(fmaf(__uint_as_float(rs[q + e]), cl2, -sd.x));
+                    if (need_mask && key > q0 + q + e) pv = 0.f;
+                    pr[e] = pv;
+                    dsr[e] = pv * (__uint_as_float(rd[q + e]) - sd.y);
+                }
+                pk[q >> 1] = pack_bf16x2(pr[0], pr[1]);
+                dk[q >> 1] = pack_bf16x2(dsr[0], dsr[1]);
+            }
+            tmem_st32(tS, pk);
+            tmem_st32(tS + 32, dk);
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(b_pfull + 8 * (n & 1));
+        }
+        const bool w = ok && mbar_wait(b_done, 0, lim, W_B_DONE, abort_flag);
+        if (__all_sync(0xffffffffu, w) && !*abort_flag) {
+            tc_fence_after_sync();
+            const size_t orow = ((size_t)kvbh * p.T + key) * D;
+            if (h == 0)
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_DK, p.scale, p.out_a + orow);  // dK
+            else
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_DV, 1.f, p.out_b + orow);  // dV
+        } else {
+            *abort_flag = 1;
+        }
+    }
+    if (warp == C::MMA_WARP && lane == 0 && *abort_flag) {
+        tc_commit(b_drain);
+        mbar_wait(b_drain, 0, lim, W_B_DRAIN);
     }
     tc_fence_before_sync();
     __syncthreads();
