@@ -63,13 +63,12 @@ def load_library():
     lib.attn_selftest_last_wait_site.argtypes = []
     lib.attn_selftest_set_exp_split.argtypes = [I]
     lib.attn_selftest_decode_plan.argtypes = [I, I, I, I, I, I, I, P, I, P, I, P, P]
-    lib.attn_selftest_set_key_tile.argtypes = [I]
     lib.attn_selftest_fused_plan.argtypes = [I, I, I, I, I, I, P, I, P]
     for name in ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_fwd_decode", "attn_fwd_unfused", "attn_fwd_host", "attn_last_error",
                  "attn_fused_grid_ctas", "attn_selftest_qk_tile", "attn_selftest_pv_tile",
                  "attn_selftest_timeout", "attn_selftest_set_mma_order",
                  "attn_selftest_last_wait_site", "attn_selftest_set_exp_split",
-                 "attn_selftest_decode_plan", "attn_selftest_set_key_tile",
+                 "attn_selftest_decode_plan",
                  "attn_selftest_fused_plan"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -307,15 +306,6 @@ def decode_plan(B: int, H: int, H_kv: int, Tq: int, Tk: int, splits: int, sms: i
     assert n2 == n
     return ([tuple(segs[8 * i:8 * i + 8]) for i in range(n)], list(nseg[:heads]), slots.value,
             copies.value)
-
-
-def set_key_tile(keys: int) -> int:
-    """Key tile of the fused forward (64 or 128; 0 = default).  Returns the
-    previous setting."""
-    prev = load_library().attn_selftest_set_key_tile(int(keys))
-    if prev == -1:
-        raise ValueError("key tile must be 0, 64 or 128")
-    return prev
 
 
 def fused_grid_ctas(B: int, H: int, T: int, D: int, causal: bool) -> int:

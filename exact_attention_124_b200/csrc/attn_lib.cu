@@ -13,7 +13,6 @@
 #include "attn.h"
 #include "attn_selftest.h"
 #include "backward.cuh"
-#include "fused_fwd_k64.cuh"
 #include "decode.cuh"
 #include "fused_fwd.cuh"
 #include "selftest.cuh"
@@ -27,34 +26,81 @@ constexpr int kMaxDevices = 64;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_mma_order = 0;
 int g_exp_split = -1;  // pairs of every 8 on the FMA pipe; -1: per-head-size default
-int g_key_tile = 0;    // fused forward key tile: 64 or 128; 0: per-head-size default
-constexpr int kDefaultKeyTile64 = 128, kDefaultKeyTile128 = 128;
 constexpr int kDefaultSplit64 = 0, kDefaultSplit128 = 0;  // measured fastest on B200
 unsigned int g_last_where = 0;
 
+// Per-device state is tied to the CUDA context it was set up in: kernel
+// attributes, the library's streams and events and the static workspace's
+// device address all die with the context (cudaDeviceReset, or any teardown
+// of the primary context), so every entry point compares the current
+// context's process-unique id with the recorded one and sets up again on a
+// mismatch.  Handles of a destroyed context are dropped, never used.
 struct DeviceState {
     bool ready = false;
+    unsigned long long ctx_id = 0;
     int sms = 0;
+    void *noalloc_ws = nullptr;  // device address of the static workspace, looked up once
 };
 DeviceState g_dev[kMaxDevices];
+
+using PfnCtxGetCurrent = CUresult (*)(CUcontext *);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long *);
+PfnCtxGetCurrent g_ctx_get_current = nullptr;
+PfnCtxGetId g_ctx_get_id = nullptr;
+
+template <typename F>
+bool driver_fn(const char *name, F &out)
+{
+    if (out) return true;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    out = reinterpret_cast<F>(fn);
+    return true;
+}
+
+// Process-unique id of the current device's context (creating the primary
+// context if none is current yet); 0 on failure.
+unsigned long long current_ctx_id()
+{
+    if (cudaFree(nullptr) != cudaSuccess) {  // makes the runtime bind its primary context
+        (void)cudaGetLastError();
+        return 0;
+    }
+    if (!driver_fn("cuCtxGetCurrent", g_ctx_get_current) || !driver_fn("cuCtxGetId", g_ctx_get_id))
+        return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        g_ctx_get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 // attn_fwd_host's copy pipeline: two non-blocking streams (host -> device,
 // device -> host) and events per chunk, created on first use per device.
 constexpr int kHostChunks = 8;
 struct HostPipe {
     bool ready = false;
+    unsigned long long ctx_id = 0;
     cudaStream_t in = nullptr, out = nullptr;
     cudaEvent_t start = nullptr, done = nullptr;
     cudaEvent_t loaded[kHostChunks] = {}, computed[kHostChunks] = {};
 };
 HostPipe g_pipe[kMaxDevices];
 
+// Called after device_ready(), which has checked the device and context.
 HostPipe *host_pipe()
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     HostPipe &hp = g_pipe[dev];
-    if (hp.ready) return &hp;
+    if (hp.ready && hp.ctx_id == g_dev[dev].ctx_id) return &hp;
+    hp = HostPipe{};  // a previous context's handles are gone with it
     bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
               cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
               cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
@@ -66,6 +112,7 @@ HostPipe *host_pipe()
         (void)cudaGetLastError();
         return nullptr;
     }
+    hp.ctx_id = g_dev[dev].ctx_id;
     hp.ready = true;
     return &hp;
 }
@@ -107,24 +154,15 @@ bool fused_ready()
 }
 
 template <int D>
-bool fused_k64_ready()
-{
-    using C = attn::FusedK64Cfg<D>;
-    if (!set_smem(attn::attn_fwd_fused_k64_kernel<D>, C::SMEM)) return false;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn::attn_fwd_fused_k64_kernel<D>) != cudaSuccess) return false;
-    return fa.numRegs >= C::REGS_LAUNCH && fa.maxThreadsPerBlock >= C::THREADS;
-}
-
-template <int D>
 bool fused_all_ready()
 {
     return fused_ready<D, 0>() && fused_ready<D, 2>() && fused_ready<D, 3>() &&
-           fused_ready<D, 4>() && fused_k64_ready<D>();
+           fused_ready<D, 4>();
 }
 
-// Per-device one-time set-up: device check (compute capability 10.0),
-// SM count, shared-memory opt-in of every kernel.
+// Per-device, per-context set-up: device check (compute capability 10.0),
+// SM count, shared-memory opt-in of every kernel.  Runs again when the
+// device's context has changed since the last set-up.
 int device_ready(int *sms_out)
 {
     int dev = -1;
@@ -132,8 +170,11 @@ int device_ready(int *sms_out)
         (void)cudaGetLastError();
         return ATTN_ERR_NO_DEVICE;
     }
+    const unsigned long long ctx = current_ctx_id();
+    if (ctx == 0) return ATTN_ERR_NO_DEVICE;
     DeviceState &st = g_dev[dev];
-    if (!st.ready) {
+    if (!st.ready || st.ctx_id != ctx) {
+        st = DeviceState{};
         int major = 0, minor = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -144,7 +185,6 @@ int device_ready(int *sms_out)
         if (major != 10 || minor != 0 || sms < 1) return ATTN_ERR_NO_DEVICE;
         if (get_encoder() != ATTN_OK) return ATTN_ERR_LAUNCH;
         bool ok = true;
-        ok &= set_smem(attn::bwd_dkdv_kernel<64>, attn::BwdCfg<64>::SMEM);
         ok &= set_smem(attn::bwd_dkdv64_kernel, attn::Dkdv64Cfg::SMEM);
         ok &= set_smem(attn::bwd_dkdv_kernel<128>, attn::BwdCfg<128>::SMEM);
         ok &= set_smem(attn::bwd_dq_kernel<64>, attn::DqCfg<64>::SMEM);
@@ -170,6 +210,7 @@ int device_ready(int *sms_out)
             return ATTN_ERR_LAUNCH;
         }
         st.sms = sms;
+        st.ctx_id = ctx;
         st.ready = true;
     }
     if (sms_out) *sms_out = st.sms;
@@ -193,6 +234,8 @@ int make_map(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uin
 }
 
 bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+// lse is read and written one float at a time: 4-byte alignment suffices.
+bool misaligned_f32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) != 0; }
 
 // Host-side checks shared by every forward entry point; no CUDA call here.
 int validate(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
@@ -203,7 +246,7 @@ int validate(const void *q, const void *k, const void *v, const void *o, const v
     if (B < 1 || H < 1 || T < 1) return ATTN_ERR_BAD_SHAPE;
     const long long bh = (long long)B * H;
     if (bh * (long long)T > (long long)INT_MAX || T > INT_MAX - 256) return ATTN_ERR_BAD_SHAPE;
-    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse))
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned_f32(lse))
         return ATTN_ERR_ALIGN;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_BAD_SCALE;
     if (causal != 0 && causal != 1) return ATTN_ERR_BAD_ARG;
@@ -259,15 +302,6 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     const int grid = fused_grid(BH, T, causal, sms);
-    const int key_tile = g_key_tile > 0 ? g_key_tile : (D == 64 ? kDefaultKeyTile64 : kDefaultKeyTile128);
-    if (key_tile == 64) {  // 64-key tiles, two score buffers per query tile (all exps on MUFU)
-        using C64 = attn::FusedK64Cfg<D>;
-        if (make_map(&mk, k, D, T, (uint64_t)B * H_kv, 64) ||
-            make_map(&mv, v, D, T, (uint64_t)B * H_kv, 64))
-            return ATTN_ERR_LAUNCH;
-        attn::attn_fwd_fused_k64_kernel<D><<<grid, C64::THREADS, C64::SMEM, stream>>>(mq, mk, mv, p);
-        return launch_status();
-    }
     const int split = g_exp_split >= 0 ? g_exp_split : (D == 64 ? kDefaultSplit64 : kDefaultSplit128);
     switch (split) {
         case 0: attn::attn_fwd_fused_kernel<D, 0><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
@@ -335,7 +369,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.limit_ns = kWaitLimitNs;
     p.out_a = static_cast<__nv_bfloat16 *>(dk);
     p.out_b = static_cast<__nv_bfloat16 *>(dv);
-    if (D == 64)  // room for 128-wide score MMAs and two S^T buffers at d_h = 64
+    if constexpr (D == 64)  // room for 128-wide score MMAs and two S^T buffers at d_h = 64
         attn::bwd_dkdv64_kernel<<<dim3(T / 128, BHkv), attn::Dkdv64Cfg::THREADS, attn::Dkdv64Cfg::SMEM,
                                   stream>>>(mq, mk, mv, mg, p);
     else
@@ -611,17 +645,18 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, vo
                 cudaMemcpyHostToDevice, hp->in) &&
              cudaEventRecord(hp->loaded[c], hp->in) == cudaSuccess;
     }
+    int fail = ATTN_OK;
     for (int c = 0; ok && c < nch; ++c) {
         const int h0 = c * per, nh = (h0 + per <= bh ? per : bh - h0);
         if (nh <= 0) break;
         const size_t off = (size_t)h0 * head * 2, bytes = (size_t)nh * head * 2;
         const size_t loff = (size_t)h0 * T * sizeof(float), lbytes = (size_t)nh * T * sizeof(float);
         if (!(ok = cudaStreamWaitEvent(s, hp->loaded[c], 0) == cudaSuccess)) break;
-        if ((rc = attn_fwd(static_cast<const char *>(dq) + off, static_cast<const char *>(dk) + off,
-                           static_cast<const char *>(dv) + off, static_cast<char *>(do_) + off,
-                           reinterpret_cast<float *>(reinterpret_cast<char *>(dlse) + loff), 1, nh,
-                           T, d_h, causal, scale, stream)))
-            return rc;
+        if ((fail = attn_fwd(static_cast<const char *>(dq) + off, static_cast<const char *>(dk) + off,
+                             static_cast<const char *>(dv) + off, static_cast<char *>(do_) + off,
+                             reinterpret_cast<float *>(reinterpret_cast<char *>(dlse) + loff), 1, nh,
+                             T, d_h, causal, scale, stream)))
+            break;
         ok = cudaEventRecord(hp->computed[c], s) == cudaSuccess &&
              cudaStreamWaitEvent(hp->out, hp->computed[c], 0) == cudaSuccess &&
              cp(static_cast<char *>(o_host) + off, static_cast<const char *>(do_) + off, bytes,
@@ -629,10 +664,16 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, vo
              cp(reinterpret_cast<char *>(lse_host) + loff, reinterpret_cast<const char *>(dlse) + loff,
                 lbytes, cudaMemcpyDeviceToHost, hp->out);
     }
-    // `stream` completes only after the last copy back
-    ok = ok && cudaEventRecord(hp->done, hp->out) == cudaSuccess &&
-         cudaStreamWaitEvent(s, hp->done, 0) == cudaSuccess;
-    if (!ok) {
+    // `stream` completes only after every copy queued above, on success and on
+    // failure alike, so the caller's buffers are not in use once it has
+    // drained (a wait uses the event's most recent record at the time of the
+    // call, so one event serves both streams in turn)
+    const bool joined = cudaEventRecord(hp->done, hp->in) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->done, 0) == cudaSuccess &&
+                        cudaEventRecord(hp->done, hp->out) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->done, 0) == cudaSuccess;
+    if (fail != ATTN_OK) return fail;
+    if (!ok || !joined) {
         (void)cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }
@@ -664,7 +705,7 @@ const char *attn_status_str(int status)
         case ATTN_ERR_NULL: return "null pointer";
         case ATTN_ERR_UNSUPPORTED_DH: return "unsupported head dimension (64 or 128)";
         case ATTN_ERR_BAD_SHAPE: return "bad shape";
-        case ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ATTN_ERR_ALIGN: return "pointer under-aligned (tensors 16 bytes, lse 4 bytes)";
         case ATTN_ERR_BAD_SCALE: return "scale not finite and positive";
         case ATTN_ERR_LAUNCH: return "CUDA launch or runtime error";
         case ATTN_ERR_TIMEOUT: return "device wait timed out";
@@ -745,14 +786,6 @@ int attn_selftest_set_mma_order(int mode)
 }
 
 int attn_selftest_last_wait_site(void) { return (int)g_last_where; }
-
-int attn_selftest_set_key_tile(int keys)
-{
-    if (keys != 0 && keys != 64 && keys != 128) return -1;
-    const int prev = g_key_tile;
-    g_key_tile = keys;
-    return prev;
-}
 
 int attn_selftest_fused_plan(int B, int H, int H_kv, int T, int causal, int sms, int *units,
                              int cap, int *ctas)
@@ -835,10 +868,6 @@ int attn_selftest_set_exp_split(int pairs_of_8)
 constexpr size_t kNoallocBytes = (size_t)64 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_ws[kNoallocBytes];
 
-namespace {
-void *g_noalloc_dev_ptr[kMaxDevices] = {};
-}
-
 extern "C" int attn_fwd_unfused_noalloc(const void *q, const void *k, const void *v, void *o,
                                         float *lse, int B, int H, int T, int d_h, int causal,
                                         float scale, void *stream)
@@ -854,15 +883,16 @@ extern "C" int attn_fwd_unfused_noalloc(const void *q, const void *k, const void
         (void)cudaGetLastError();
         return ATTN_ERR_NO_DEVICE;
     }
-    if (g_noalloc_dev_ptr[dev] == nullptr) {  // first call on this device
+    DeviceState &st = g_dev[dev];
+    if (st.noalloc_ws == nullptr) {  // first call on this device (in this context)
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_ws) != cudaSuccess || ptr == nullptr) {
             (void)cudaGetLastError();
             return ATTN_ERR_LAUNCH;
         }
-        g_noalloc_dev_ptr[dev] = ptr;
+        st.noalloc_ws = ptr;
     }
-    auto *ws = static_cast<unsigned char *>(g_noalloc_dev_ptr[dev]);
+    auto *ws = static_cast<unsigned char *>(st.noalloc_ws);
     void *s_ws = ws;
     void *p_ws = ws + kNoallocBytes / 2;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const BwdParams p)
 {
+    static_assert(D == 128, "d_h = 64 runs bwd_dkdv64_kernel");
     using C = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     BwdSmem<D> sm;

@@ -332,6 +332,7 @@ __global__ void __launch_bounds__(192, 1)
             const int pos = p.Tk - p.Tq + qi;
             const int lim_key = p.causal ? pos : p.Tk - 1;
             float m = -INFINITY, l = 0.f;
+            float lcor = 0.f;  // bf16 rounding of each tile's largest weight (normaliser of O only)
             for (int j = 0; ok && j < n; ++j) {
                 const uint32_t t = u + j;
                 const int buf = t & 1;
@@ -391,7 +392,12 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
                 l *= alpha;
+                lcor *= alpha;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                {  // the P.V MMA sees bf16 weights; see the fused kernel's softmax
+                    const float pmax = fast_exp2(fmaf(mx, cl2, neg_m));
+                    lcor += bf16_round(pmax) - pmax;
+                }
                 float ls = 0.f;
                 // P over the first 64 S columns (bf16 pairs): this copy's W keys
                 // at pair columns [cp W / 2, cp W / 2 + W / 2), zeros elsewhere
@@ -435,7 +441,7 @@ __global__ void __launch_bounds__(192, 1)
             const size_t row = (size_t)(b * p.H + kvl * p.group + g) * p.Tq + qi;
             // each copy's result is one more partial of this row
             const size_t at = ((size_t)sg.slot * CP + cp) * (size_t)p.nrows + row;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = l > 0.f ? 1.f / (l + lcor) : 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t rg[32];

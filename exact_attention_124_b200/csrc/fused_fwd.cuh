@@ -513,7 +513,8 @@ __global__ void __launch_bounds__(384, 1)
             const int r0 = u.i0 + 128 * t;
             const int row = r0 + rit;
             float m = -INFINITY;  // running max, log2 units
-            float l = 0.f;        // running normaliser
+            float l = 0.f;        // running normaliser (fp32 weights)
+            float lcor = 0.f;     // bf16 rounding of each tile's largest weight
             for (int j = 0; j < nt; ++j) {
                 bool w = mbar_wait(b_sfull + 8 * t, sph, lim, W_SFULL, abort_flag);
                 ok = __all_sync(0xffffffffu, w);
@@ -536,7 +537,8 @@ __global__ void __launch_bounds__(384, 1)
                     for (int c = 0; c < 128; ++c)
                         if (key0 + c > lim_key) s[c] = -INFINITY;
                 }
-                const float cand = row_max(s) * cl2;
+                const float smax = row_max(s);
+                const float cand = smax * cl2;
                 float alpha = 1.f;
                 bool resc = false;
                 if (j == 0) {
@@ -559,6 +561,7 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
                 l *= alpha;
+                lcor *= alpha;
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const float2 c2 = make_float2(cl2, cl2);
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -584,6 +587,14 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_before_sync();
                 mbar_arrive(b_pfull + 16 * t + 8);  // keys 64-127
                 l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+                // The P.V MMA multiplies bf16-rounded weights while l sums the
+                // fp32 ones.  On a row dominated by one key that mismatch would
+                // scale O by up to 1 +- 2^-9; the dominant key is its tile's
+                // largest score, so the normaliser of O takes that element's
+                // rounding error (its p recomputed bit for bit: the same fma
+                // and ex2 as above).  lse keeps the fp32 sum.
+                const float pmax = fast_exp2(fmaf(smax, cl2, neg_m));
+                lcor += bf16_round(pmax) - pmax;
             }
             if (!ok) break;
             // epilogue: O = acc / l, lse = (m + log2 l) ln 2
@@ -592,7 +603,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             oph ^= 1u;
             tc_fence_after_sync();
-            const float inv_l = 1.f / l;
+            const float inv_l = 1.f / (l + lcor);
             const size_t orow = (size_t)u.bh * (size_t)p.T + (size_t)row;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {

@@ -359,6 +359,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// x rounded to bf16 (nearest even), as fp32.
+__device__ __forceinline__ float bf16_round(float x)
+{
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ float fast_exp2(float x)
 {
     float y;

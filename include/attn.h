@@ -17,9 +17,15 @@
  *  - Layout: q, k, v, o are bf16, [B, H, T, d_h] contiguous (row = token,
  *    d_h values contiguous); lse is fp32, [B, H, T].  Head (b, h) starts at
  *    element ((b * H + h) * T) * d_h.
- *  - Pointers are device pointers unless the name says host; all must be
- *    16-byte aligned (tensor-memory-accelerator rule).  The caller owns all
+ *  - Pointers are device pointers unless the name says host.  Tensor and
+ *    workspace pointers must be 16-byte aligned (tensor-memory-accelerator
+ *    rule); lse pointers need only float (4-byte) alignment, since every
+ *    kernel reads and writes lse one value at a time.  The caller owns all
  *    memory; no entry point allocates device memory.
+ *  - Per-device set-up (kernel attributes, the library's own streams and
+ *    events, the static workspace's address) is done on the first call in a
+ *    CUDA context and redone when the device's current context changes (for
+ *    example after cudaDeviceReset), so no handle outlives its context.
  *  - d_h must be 64 or 128.  B, H, T >= 1.  B * H * T must fit in 2^31 - 1
  *    and T in 2^31 / 256.  scale must be finite and > 0 (configs use
  *    1 / sqrt(d_h)).  causal is 0 or 1 (top-left aligned, Tq = Tk = T).
@@ -45,7 +51,7 @@ typedef enum {
     ATTN_ERR_NULL = 1,           /* a required pointer is NULL                         */
     ATTN_ERR_UNSUPPORTED_DH = 2, /* d_h not in {64, 128}                               */
     ATTN_ERR_BAD_SHAPE = 3,      /* B, H or T < 1, or sizes overflow the limits above  */
-    ATTN_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned                   */
+    ATTN_ERR_ALIGN = 4,          /* a pointer is under-aligned (see the conventions)   */
     ATTN_ERR_BAD_SCALE = 5,      /* scale not finite or <= 0                           */
     ATTN_ERR_LAUNCH = 6,         /* a CUDA runtime/driver call failed                  */
     ATTN_ERR_TIMEOUT = 7,        /* device: a bounded wait ran out; the kernel returned */

@@ -72,16 +72,6 @@ int attn_selftest_set_exp_split(int pairs_of_8);
 int attn_selftest_last_wait_site(void);
 
 /*
- * Key tile of the fused forward: 128 (P written over the score tile; the
- * exp-split variants apply) or 64 (two score buffers per query tile, the next
- * score MMA overlapping the softmax; all exponentials on MUFU); 0 restores
- * the per-head-size default.  Same arithmetic up to the order of the online
- * softmax's rescaling.  Returns the previous setting (0 = default), or -1 for
- * another value.
- */
-int attn_selftest_set_key_tile(int keys);
-
-/*
  * Host only (no device needed): the work units the fused forward would run
  * for these sizes on a device with `sms` SMs, computed by the kernel's own
  * unit function.  A unit is 256 query rows of one query head: two 128-row

@@ -1,6 +1,6 @@
 """Seeded random shapes through every GPU entry point, each checked against
 the float64 oracle with the bar of its own parity tests: grouped-query
-forward (any T, both d_h, causal or not, both key tiles), backward (T a
+forward (any T, both d_h, causal or not), backward (T a
 multiple of 128, long enough for the K/V rings to wrap several times) and
 decode (fixed, balanced and automatic partitions, 1, 2 or 4 row copies)."""
 import math
@@ -30,24 +30,20 @@ def _fwd_cases(n=16, seed=424242):
     for i in range(n):
         H_kv = rng.randint(1, 3)
         out.append((rng.randint(1, 2), H_kv * rng.randint(1, 3), H_kv, rng.randint(1, 700),
-                    rng.choice([64, 128]), rng.random() < 0.6, rng.choice([64, 128]), 31000 + i))
+                    rng.choice([64, 128]), rng.random() < 0.6, 31000 + i))
     return out
 
 
-@pytest.mark.parametrize("B,H,H_kv,T,D,causal,key_tile,seed", _fwd_cases())
-def test_random_forward(B, H, H_kv, T, D, causal, key_tile, seed):
+@pytest.mark.parametrize("B,H,H_kv,T,D,causal,seed", _fwd_cases())
+def test_random_forward(B, H, H_kv, T, D, causal, seed):
     q, _, _ = make_qkv(B, H, T, D, seed)
     _, k, v = make_qkv(B, H_kv, T, D, seed + 500)
-    prev = attn.set_key_tile(key_tile)
-    try:
-        o, lse = attn.fwd_gqa(*to_dev(q, k, v), causal)
-    finally:
-        attn.set_key_tile(prev)
+    o, lse = attn.fwd_gqa(*to_dev(q, k, v), causal)
     assert attn.last_error() == 0
     ro, rl = oracle.attn_fwd_gqa(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 1 / math.sqrt(D))
     st = compare(o.double().cpu().numpy().reshape(ro.shape),
                  lse.double().cpu().numpy().reshape(rl.shape), ro, rl)
-    assert_parity(st, f"fwd B={B} H={H} H_kv={H_kv} T={T} D={D} causal={causal} kt={key_tile}")
+    assert_parity(st, f"fwd B={B} H={H} H_kv={H_kv} T={T} D={D} causal={causal}")
 
 
 BWD_CASES = [(1, 2, 1, 2048, 128, True, 32001), (1, 2, 2, 1536, 64, False, 32002),
