@@ -38,7 +38,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_inputs import WORKLOADS, make_qkv, bf16_bits  # noqa: E402
+from attn_inputs import ORDER, WORKLOADS, make_qkv, bf16_bits  # noqa: E402
 
 DEFAULT_WORKLOAD = "causal_T8192_d128"
 METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other workloads (the per_config block)")
     ap.add_argument("--decode-tq", type=int, default=1, help="decode: new queries per head")
     ap.add_argument("--decode-hkv", type=int, default=0,
                     help="decode: K/V heads (0: the workload's H / 4)")
@@ -69,9 +71,6 @@ def parse():
     ap.add_argument("--exp-split", type=int, default=None,
                     help="fused kernel variant: column pairs of every 8 whose exponentials run "
                          "on the FMA pipe (0, 2, 3, 4); default: the library's choice")
-    ap.add_argument("--key-tile", type=int, default=None, choices=[64, 128],
-                    help="fused kernel variant: key tile 64 (two score buffers per query tile) "
-                         "or 128; default: the library's choice")
     args = ap.parse_args()
     if args.e2e_steps < 1 or args.steps < 1:
         ap.error("--steps and --e2e-steps must be at least 1")
@@ -302,8 +301,6 @@ def run_ours(args):
     attn.load_library()
     if args.exp_split is not None:
         attn.set_exp_split(args.exp_split)
-    if args.key_tile is not None:
-        attn.set_key_tile(args.key_tile)
     peaks, peak_src = load_peaks()
     other = {"unfused": run_unfused, "backward": run_backward, "decode": run_decode}.get(args.path)
     if other is not None:
@@ -320,38 +317,25 @@ def run_ours(args):
     lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        attn.fwd(qd, kd, vd, w.causal, w.scale, o=o, lse=lse, stream=stream)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    if attn.last_error() != 0:
-        raise SystemExit("device error during warm-up")
-
-    # timed region: events around every launch on the launching stream
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    sampler = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    ev[0].record(stream)
-    for i in range(args.steps):
-        step()
-        ev[i + 1].record(stream)
-    torch.cuda.synchronize()
-    sampler.stop()
-    if world > 1:
-        dist.barrier()
+    per_launch, total_ms, clocks_main = time_fused(attn, w, qd, kd, vd, o, lse, stream, args.steps,
+                                                   args.warmup, local, world)
     status = attn.last_error()
     launches = args.steps  # one fused kernel per step
-    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
     ms = max_over_ranks(total_ms / args.steps, world, dev)
     flops = counted_flops(w)
     value = whole_job_tflops(flops, world, ms)
     achieved = flops / (statistics.mean(per_launch) * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
+
+    # the other workloads, timed the same way on this GPU (rank 0 at N = 1 only)
+    per_config = None
+    if world == 1 and not args.no_per_config and args.workload == DEFAULT_WORKLOAD:
+        per_config = {}
+        for name in ORDER:
+            if name == w.name:
+                continue
+            per_config[name] = time_other(attn, WORKLOADS[name], dev, stream, args, local, peaks)
+            status |= attn.last_error()
 
     # end to end through the host-buffer C-ABI entry point
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
@@ -381,7 +365,7 @@ def run_ours(args):
                "sample": desc, "seconds": round(dt, 2)}
 
     if rank == 0:
-        clocks = sampler.summary()
+        clocks = clocks_main
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -406,6 +390,7 @@ def run_ours(args):
                          "launch_ms_mean": statistics.mean(per_launch),
                          "launch_ms_min": min(per_launch)},
             "clocks": clocks,
+            "per_config": per_config,
             "gpu_launches": launches,
             "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -418,6 +403,70 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0 if status == 0 else 1
+
+
+def time_fused(attn, w, qd, kd, vd, o, lse, stream, steps, warmup, local, world, flush=None):
+    """W untimed launches, then K launches with CUDA events around each on the
+    launching stream and NVML clock sampling meanwhile.  With ``flush`` (a
+    device buffer larger than L2) the buffer is rewritten before every launch,
+    outside the events.  Returns (per-launch ms, first-to-last ms, clocks)."""
+    import torch
+    import torch.distributed as dist
+
+    def step():
+        attn.fwd(qd, kd, vd, w.causal, w.scale, o=o, lse=lse, stream=stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    if attn.last_error() != 0:
+        raise SystemExit(f"device error during warm-up ({w.name})")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        ev[2 * i].record(stream)
+        step()
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if world > 1:
+        dist.barrier()
+    per_launch = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
+    total = ev[0].elapsed_time(ev[-1]) if flush is None else sum(per_launch)
+    return per_launch, total, sampler.summary()
+
+
+def time_other(attn, w, dev, stream, args, local, peaks):
+    """One entry of the bench line's per_config block: workload ``w`` timed
+    like the headline (inputs resident; L2 rewritten before each launch when
+    the inputs would fit in it)."""
+    import torch
+    q, k, v = make_qkv(w.B, w.H, w.T, w.D, w.seed, w.qk_mult)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    del q, k, v
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+    in_bytes = 3 * qd.numel() * 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < (256 << 20) else None
+    per_launch, _, clocks = time_fused(attn, w, qd, kd, vd, o, lse, stream, args.steps,
+                                       args.warmup, local, 1, flush)
+    mean_ms = statistics.mean(per_launch)
+    tf = counted_flops(w) / (mean_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    out = {"shape": w.describe(), "seed": w.seed, "ms_mean": mean_ms, "ms_min": min(per_launch),
+           "tflops": tf, "frac": tf / peak, "frac_of_datasheet_2250": tf / 2250.0,
+           "l2": ("256 MB rewritten before each launch" if flush is not None else
+                  "inputs larger than L2 (%.0f MB); no flush" % (in_bytes / 1e6)),
+           "grid_ctas": attn.fused_grid_ctas(w.B, w.H, w.T, w.D, w.causal), "launches": args.steps,
+           "clocks": clocks}
+    del qd, kd, vd, o, lse, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def unfused_bytes(w) -> int:
