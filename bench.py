@@ -537,13 +537,12 @@ def run_backward(args, w, world, rank, local, peaks, peak_src):
     import torch
     import exact_attention_124_b200 as attn
     dev = torch.device("cuda", local)
-    if w.T % 128:
-        raise SystemExit("the backward pass needs T to be a multiple of 128")
     q, k, v = [t.to(dev) for t in make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank), w.qk_mult)]
     g = make_qkv(w.B, w.H, w.T, w.D, rank_seed(w, rank) + 7)[0].to(dev)
     o, lse = attn.fwd(q, k, v, w.causal, w.scale)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(w.B * w.H * w.T * 8, dtype=torch.uint8, device=dev)
+    ws = torch.empty(int(attn.load_library().attn_bwd_workspace_bytes(w.B, w.H, w.T)),
+                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():

@@ -351,10 +351,11 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         make_map(&mk, k, D, T, BHkv, 128) || make_map(&mv, v, D, T, BHkv, 128))
         return ATTN_ERR_LAUNCH;
     auto *stats = static_cast<float2 *>(ws);
-    const long long rows = (long long)BH * T;
-    attn::bwd_stats_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+    const int nq = (T + 127) / 128, Tp = 128 * nq;  // a ragged last block is padded
+    const long long prow = (long long)BH * Tp;
+    attn::bwd_stats_kernel<D><<<(unsigned)((prow + 7) / 8), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse,
-        stats, rows);
+        stats, prow, T, Tp);
     if (launch_status()) return ATTN_ERR_LAUNCH;
     attn::BwdParams p;
     p.stats = stats;
@@ -362,7 +363,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.H_kv = H_kv;
     p.group = H / H_kv;
     p.T = T;
-    p.nq = T / 128;
+    p.nq = nq;
+    p.Tp = Tp;
     p.causal = causal;
     p.c_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
@@ -370,15 +372,15 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.out_a = static_cast<__nv_bfloat16 *>(dk);
     p.out_b = static_cast<__nv_bfloat16 *>(dv);
     if constexpr (D == 64)  // room for 128-wide score MMAs and two S^T buffers at d_h = 64
-        attn::bwd_dkdv64_kernel<<<dim3(T / 128, BHkv), attn::Dkdv64Cfg::THREADS, attn::Dkdv64Cfg::SMEM,
+        attn::bwd_dkdv64_kernel<<<dim3(nq, BHkv), attn::Dkdv64Cfg::THREADS, attn::Dkdv64Cfg::SMEM,
                                   stream>>>(mq, mk, mv, mg, p);
     else
-        attn::bwd_dkdv_kernel<D><<<dim3(T / 128, BHkv), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
+        attn::bwd_dkdv_kernel<D><<<dim3(nq, BHkv), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mg, p);
     if (launch_status()) return ATTN_ERR_LAUNCH;
     p.out_a = static_cast<__nv_bfloat16 *>(dq);
     p.out_b = nullptr;
     using Q = attn::DqCfg<D>;
-    attn::bwd_dq_kernel<D><<<dim3(T / 128, BH), Q::THREADS, Q::SMEM, stream>>>(mq, mk, mv, mg, p);
+    attn::bwd_dq_kernel<D><<<dim3(nq, BH), Q::THREADS, Q::SMEM, stream>>>(mq, mk, mv, mg, p);
     return launch_status();
 }
 
@@ -538,8 +540,9 @@ int attn_fwd_decode(const void *q, const void *k, const void *v, void *o, float 
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T)
 {
-    if (B < 1 || H < 1 || T < 1) return 0;
-    return (size_t)B * H * T * 8;
+    if (B < 1 || H < 1 || T < 1 || T > INT_MAX - 128) return 0;
+    const size_t Tp = (size_t)((T + 127) / 128) * 128;  // per-row statistics, 128-row blocks
+    return (size_t)B * H * Tp * 8;
 }
 
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -551,7 +554,8 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const f
     if (!dout || !dq || !dk || !dv || !ws) return ATTN_ERR_NULL;
     if (misaligned(dout) || misaligned(dq) || misaligned(dk) || misaligned(dv) || misaligned(ws))
         return ATTN_ERR_ALIGN;
-    if (H_kv < 1 || H % H_kv != 0 || T % 128 != 0 || (long long)B * H > 65535)
+    if (H_kv < 1 || H % H_kv != 0 || (long long)B * H > 65535 ||
+        (long long)B * H * (((long long)T + 127) / 128 * 128) > (long long)INT_MAX)
         return ATTN_ERR_BAD_SHAPE;
     if ((rc = device_ready(nullptr))) return rc;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);

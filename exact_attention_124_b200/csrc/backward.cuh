@@ -35,10 +35,11 @@
 namespace attn {
 
 struct BwdParams {
-    const float2 *stats;  // [B*H, T] (lse * log2 e, D)
+    const float2 *stats;  // [B*H, Tp] (lse * log2 e, D); rows T .. Tp-1 of a head: (+inf, 0)
     __nv_bfloat16 *out_a; // dkdv: dK [B*H_kv, T, D];  dq: dQ [B*H, T, D]
     __nv_bfloat16 *out_b; // dkdv: dV [B*H_kv, T, D]
     int H, H_kv, group, T, nq, causal;
+    int Tp;               // T rounded up to the 128-row block: 128 * nq
     float c_log2;         // scale * log2 e
     float scale;
     unsigned long long limit_ns;
@@ -71,15 +72,26 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------- preprocess
-// stats[r] = (lse[r] * log2 e, sum_c dO[r][c] O[r][c]); one warp per row.
+// stats[h * Tp + t] = (lse * log2 e, sum_c dO[c] O[c]) of row t of head h, one
+// warp per row; rows t >= T (padding up to the 128-row block) get (+inf, 0):
+// their probabilities 2^(s - inf) are exactly 0 and their dS = P (dP - 0) too,
+// so the zero rows the tensor maps read there add nothing to the gradients.
 template <int D>
 __global__ void __launch_bounds__(256)
     bwd_stats_kernel(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
-                     const float *__restrict__ lse, float2 *__restrict__ stats, long long rows)
+                     const float *__restrict__ lse, float2 *__restrict__ stats, long long prow,
+                     int T, int Tp)
 {
-    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long pr = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (r >= rows) return;
+    if (pr >= prow) return;
+    const long long head = pr / Tp;
+    const int t = (int)(pr - head * Tp);
+    if (t >= T) {
+        if (lane == 0) stats[pr] = make_float2(INFINITY, 0.f);
+        return;
+    }
+    const long long r = head * T + t;
     constexpr int PER = D / 32;  // bf16 values per lane: 4 (8 bytes) or 2 (4 bytes)
     const __nv_bfloat16 *o = O + r * D + lane * PER;
     const __nv_bfloat16 *g = dO + r * D + lane * PER;
@@ -88,7 +100,7 @@ __global__ void __launch_bounds__(256)
     for (int i = 0; i < PER; ++i) acc = fmaf(__bfloat162float(o[i]), __bfloat162float(g[i]), acc);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) stats[r] = make_float2(lse[r] * 1.4426950408889634f, acc);
+    if (lane == 0) stats[pr] = make_float2(lse[r] * 1.4426950408889634f, acc);
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
@@ -212,9 +224,11 @@ __device__ __forceinline__ void bwd_elementwise(uint32_t tS, uint32_t tDP, float
 }
 
 // Epilogue: 32-column chunks [C0, C1) of the rows of a TMEM accumulator times
-// `mul`, as bf16.
+// `mul`, as bf16; a lane whose row is padding (`store` false) reads its TMEM
+// lane like the others -- tcgen05.ld is a whole-warp instruction -- and writes
+// nothing.
 template <int C0, int C1>
-__device__ __forceinline__ void store_rows(uint32_t tacc, float mul, __nv_bfloat16 *dst)
+__device__ __forceinline__ void store_rows(uint32_t tacc, float mul, __nv_bfloat16 *dst, bool store)
 {
 #pragma unroll
     for (int c = C0; c < C1; ++c) {
@@ -225,10 +239,12 @@ __device__ __forceinline__ void store_rows(uint32_t tacc, float mul, __nv_bfloat
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
-        uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+        if (store) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
     }
 }
 
@@ -324,7 +340,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                     tma_load_3d(st + C::TILE + kb * C::SUB, &tmdO, sm.b_full + 8 * s, 64 * kb,
                                 128 * i, bh, pol);
                 }
-                bulk_load(st + 2 * C::TILE, p.stats + (size_t)bh * p.T + 128 * i, 1024,
+                bulk_load(st + 2 * C::TILE, p.stats + (size_t)bh * p.Tp + 128 * i, 1024,
                           sm.b_full + 8 * s);
             }
             if (!ok) {
@@ -401,10 +417,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (__all_sync(0xffffffffu, w) && !*sm.abort_flag) {
             tc_fence_after_sync();
             const size_t orow = ((size_t)kvbh * p.T + key) * D;
+            const bool real = key < p.T;  // padding rows of the last key block store nothing
             if (h == 0)
-                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC1, p.scale, p.out_a + orow);  // dK
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC1, p.scale, p.out_a + orow, real);  // dK
             else
-                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC0, 1.f, p.out_b + orow);  // dV
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_ACC0, 1.f, p.out_b + orow, real);  // dV
         } else {
             *sm.abort_flag = 1;
         }
@@ -530,7 +547,7 @@ __global__ void __launch_bounds__(Dkdv64Cfg::THREADS, 1)
                 armed_par = (armed_par & ~(1u << s2)) | (par << s2);
                 tma_load_3d(st, &tmQ, b_full + 8 * s2, 0, 128 * i, bh, pol);
                 tma_load_3d(st + C::TILE, &tmdO, b_full + 8 * s2, 0, 128 * i, bh, pol);
-                bulk_load(st + 2 * C::TILE, p.stats + (size_t)bh * p.T + 128 * i, 1024, b_full + 8 * s2);
+                bulk_load(st + 2 * C::TILE, p.stats + (size_t)bh * p.Tp + 128 * i, 1024, b_full + 8 * s2);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -678,10 +695,11 @@ __global__ void __launch_bounds__(Dkdv64Cfg::THREADS, 1)
         if (__all_sync(0xffffffffu, w) && !*abort_flag) {
             tc_fence_after_sync();
             const size_t orow = ((size_t)kvbh * p.T + key) * D;
+            const bool real = key < p.T;  // padding rows of the last key block store nothing
             if (h == 0)
-                store_rows<0, D / 32>(tmem + lane_off + C::TM_DK, p.scale, p.out_a + orow);  // dK
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_DK, p.scale, p.out_a + orow, real);  // dK
             else
-                store_rows<0, D / 32>(tmem + lane_off + C::TM_DV, 1.f, p.out_b + orow);  // dV
+                store_rows<0, D / 32>(tmem + lane_off + C::TM_DV, 1.f, p.out_b + orow, real);  // dV
         } else {
             *abort_flag = 1;
         }
@@ -911,7 +929,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         const int qr = (warp & 3) * 32 + lane;
         const int row = 128 * i + qr;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const float2 st = p.stats[(size_t)bh * p.T + row];
+        const float2 st = p.stats[(size_t)bh * p.Tp + row];
         const float cl2 = p.c_log2;
         bool ok = true;
         for (int n = 0; ok && n < nkb; ++n) {
@@ -965,10 +983,11 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         if (__all_sync(0xffffffffu, w) && !*abort_flag) {
             tc_fence_after_sync();
             __nv_bfloat16 *dst = p.out_a + ((size_t)bh * p.T + row) * D;
+            const bool real = row < p.T;  // padding rows of the last query block store nothing
             if (h == 0)  // the two warpgroups store the two halves of the d_h columns
-                store_rows<0, D / 64>(tmem + lane_off + C::TM_DQ, p.scale, dst);
+                store_rows<0, D / 64>(tmem + lane_off + C::TM_DQ, p.scale, dst, real);
             else
-                store_rows<D / 64, D / 32>(tmem + lane_off + C::TM_DQ, p.scale, dst);
+                store_rows<D / 64, D / 32>(tmem + lane_off + C::TM_DQ, p.scale, dst, real);
         } else {
             *abort_flag = 1;
         }

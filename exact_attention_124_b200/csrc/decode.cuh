@@ -57,7 +57,7 @@ struct DecodeParams {
     unsigned long long limit_ns;
 };
 
-constexpr float DEC_RESCALE_TAU = 8.0f;  // lazy rescale threshold, log2 units (as prefill)
+constexpr float DEC_RESCALE_TAU = 32.0f;  // lazy rescale threshold, log2 units (as prefill)
 
 enum : unsigned int {
     W_D_Q = 128, W_D_KVFULL, W_D_KVEMPTY, W_D_SFULL, W_D_PFULL, W_D_PVDONE, W_D_DRAIN, W_D_QEMPTY,

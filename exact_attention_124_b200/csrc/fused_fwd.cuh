@@ -36,20 +36,23 @@
 //   O_0       : [256, 256 + d_h)     O_1       : [256 + d_h, 256 + 2 d_h)
 // Online softmax in the log2 domain: s2 = s * scale * log2(e); the running
 // maximum m only moves when a row's new maximum exceeds it by more than
-// RESCALE_TAU (2^8 headroom keeps p <= 256), so the O rescale (a TMEM
-// read-modify-write) is rare; the final O = acc / l and lse = (m + log2 l) ln 2
-// are exact for any m, stale or not.
+// RESCALE_TAU = 32, so the O rescale (a TMEM read-modify-write of the whole
+// warp's rows, done when any of its 32 rows needs it) is rare; the final
+// O = acc / l and lse = (m + log2 l) ln 2 are exact for any m, stale or not.
+// A stale m only makes the weights larger, p <= 2^32: far inside the range of
+// bf16 P and of the fp32 O and l (2^32 x 2^31 keys x |v| < 2^127), and
+// floating point keeps its relative precision at any scale.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace attn {
 
-constexpr float RESCALE_TAU = 8.0f;
+constexpr float RESCALE_TAU = 32.0f;
 
 // 2^x on the FMA pipe for two values at once (x <= RESCALE_TAU).  Range
 // reduction x = n + f, n = round(x) (adding 1.5 * 2^23 rounds to an integer in
-// the low mantissa bits), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// the low mantissa bits, |n| < 256), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
 // coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
 // exchange, computed by gen_exp2_poly.py next to this file; max relative
 // error 7.5e-5, far below the bf16 rounding of P); 2^n by adding n to the
@@ -155,10 +158,11 @@ __device__ __forceinline__ float row_max(const float (&s)[128])
 
 // p = 2^(s * c - m) for column pairs P0 .. P0+NP-1, packed to bf16 pairs in pk;
 // the fp32 p are summed into ls (two packed accumulators).
-template <int EMU, int P0, int NP>
-__device__ __forceinline__ void exp_pairs(const float (&s)[128], float2 c2, float2 nm2,
+template <int EMU, int P0, int NP, int N>
+__device__ __forceinline__ void exp_pairs(const float (&s)[N], float2 c2, float2 nm2,
                                           uint32_t (&pk)[NP], float2 (&ls)[2])
 {
+    static_assert(2 * (P0 + NP) <= N, "pairs past the array");
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
         const int pi = P0 + i;
@@ -539,6 +543,17 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 const float smax = row_max(s);
                 const float cand = smax * cl2;
+                // Does the tile's largest score sit in a pair whose exponential the
+                // FMA pipe evaluates?  Its weight for the correction below must
+                // come from the same evaluation (variants with EMU > 0 only).
+                bool max_emu = false;
+                if constexpr (EMU > 0) {
+                    if (!need_mask) {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i)
+                            if (emu_pair<EMU>(i)) max_emu |= (s[2 * i] == smax) | (s[2 * i + 1] == smax);
+                    }
+                }
                 float alpha = 1.f;
                 bool resc = false;
                 if (j == 0) {
@@ -591,9 +606,13 @@ __global__ void __launch_bounds__(384, 1)
                 // fp32 ones.  On a row dominated by one key that mismatch would
                 // scale O by up to 1 +- 2^-9; the dominant key is its tile's
                 // largest score, so the normaliser of O takes that element's
-                // rounding error (its p recomputed bit for bit: the same fma
-                // and ex2 as above).  lse keeps the fp32 sum.
-                const float pmax = fast_exp2(fmaf(smax, cl2, neg_m));
+                // rounding error (its p recomputed bit for bit: the same fma,
+                // and the same ex2 or polynomial, as above -- two evaluations
+                // 7.5e-5 apart can round to neighbouring bf16 values, an error
+                // of 2^-8 that the correction would then add instead of
+                // removing).  lse keeps the fp32 sum.
+                const float xmax = fmaf(smax, cl2, neg_m);
+                const float pmax = max_emu ? exp2_poly2(make_float2(xmax, xmax)).x : fast_exp2(xmax);
                 lcor += bf16_round(pmax) - pmax;
             }
             if (!ok) break;

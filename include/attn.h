@@ -125,14 +125,17 @@ size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int d
  *   dq         : out, bf16 [B, H, T, d_h];  dk, dv : out, bf16 [B, H_kv, T, d_h]
  *   ws         : caller-owned device workspace of attn_bwd_workspace_bytes()
  *                bytes (per-row statistics; contents on return unspecified)
- * T must be a multiple of 128; H % H_kv == 0; B * H <= 65535.  Other
- * arguments, errors and asynchrony as attn_fwd.
+ * Any T >= 1 (a ragged last block of 128 rows is padded internally);
+ * H % H_kv == 0; B * H <= 65535; B * H * Tp < 2^31 with Tp = T rounded up to
+ * a multiple of 128.  Other arguments, errors and asynchrony as attn_fwd.
  */
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dout, void *dq, void *dk, void *dv, void *ws, int B, int H, int H_kv,
              int T, int d_h, int causal, float scale, void *stream);
 
-/* Bytes of attn_bwd's workspace: B * H * T * 8.  0 on bad sizes. */
+/* Bytes of attn_bwd's workspace: B * H * Tp * 8, Tp = T rounded up to a
+ * multiple of 128 (one pair of fp32 row statistics per padded row).  0 on bad
+ * sizes. */
 size_t attn_bwd_workspace_bytes(int B, int H, int T);
 
 /*

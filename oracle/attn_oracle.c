@@ -263,61 +263,137 @@ void oracle_head_fwd_f64(const double *q, const double *k, const double *v, int 
     free(mk);
 }
 
+/* Gradients of one head on double inputs, in two passes over independent
+ * outputs (so that the row pass and the key pass can each be split across
+ * threads without changing any output's arithmetic):
+ *   rows i:  S_i and P_i (the forward's definition), dP_i = dO_i V^T,
+ *            dS_i = P_i o (dP_i - sum_j P_ij dP_ij),  dQ_i = scale sum_j dS_ij K_j
+ *   keys j:  dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij Q_i
+ * Every sum runs over its index in ascending order. */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    int T, D, causal;
+    double scale;
+    double *P, *dS, *dq, *dk, *dv;
+    int tid, nthreads;
+} head_bwd_job_t;
+
+static void *head_bwd_rows(void *arg)
+{
+    head_bwd_job_t *jb = (head_bwd_job_t *)arg;
+    const int T = jb->T, D = jb->D;
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    double *acc = (double *)malloc(sizeof(double) * (size_t)D);
+    unsigned char *mk = (unsigned char *)malloc((size_t)T);
+    for (int i = jb->tid; i < T; i += jb->nthreads) {
+        const double *qi = jb->q + (size_t)i * D, *gi = jb->dout + (size_t)i * D;
+        double *Pi = jb->P + (size_t)i * T, *dSi = jb->dS + (size_t)i * T;
+        for (int j = 0; j < T; ++j) { /* S and P of row i */
+            double a = 0.0;
+            for (int c = 0; c < D; ++c)
+                a += qi[c] * jb->k[(size_t)j * D + c];
+            s[j] = jb->scale * a;
+            mk[j] = (unsigned char)(jb->causal && j > i);
+        }
+        oracle_softmax_row(s, mk, T, Pi);
+        for (int j = 0; j < T; ++j) { /* dP of row i, kept in dS_i for now */
+            double a = 0.0;
+            for (int c = 0; c < D; ++c)
+                a += gi[c] * jb->v[(size_t)j * D + c];
+            dSi[j] = a;
+        }
+        double r = 0.0; /* dS_i = P_i o (dP_i - rowsum(P_i o dP_i)) */
+        for (int j = 0; j < T; ++j)
+            r += Pi[j] * dSi[j];
+        for (int j = 0; j < T; ++j)
+            dSi[j] = Pi[j] * (dSi[j] - r);
+        for (int c = 0; c < D; ++c) /* dQ_i = scale sum_j dS_ij K_j */
+            acc[c] = 0.0;
+        for (int j = 0; j < T; ++j)
+            for (int c = 0; c < D; ++c)
+                acc[c] += dSi[j] * jb->k[(size_t)j * D + c];
+        for (int c = 0; c < D; ++c)
+            jb->dq[(size_t)i * D + c] = jb->scale * acc[c];
+    }
+    free(s);
+    free(acc);
+    free(mk);
+    return NULL;
+}
+
+static void *head_bwd_keys(void *arg)
+{
+    head_bwd_job_t *jb = (head_bwd_job_t *)arg;
+    const int T = jb->T, D = jb->D;
+    double *pc = (double *)malloc(sizeof(double) * (size_t)T);
+    double *sc = (double *)malloc(sizeof(double) * (size_t)T);
+    double *av = (double *)malloc(sizeof(double) * (size_t)D);
+    double *ak = (double *)malloc(sizeof(double) * (size_t)D);
+    for (int j = jb->tid; j < T; j += jb->nthreads) {
+        for (int i = 0; i < T; ++i) { /* column j of P and of dS */
+            pc[i] = jb->P[(size_t)i * T + j];
+            sc[i] = jb->dS[(size_t)i * T + j];
+        }
+        for (int c = 0; c < D; ++c)
+            av[c] = ak[c] = 0.0;
+        for (int i = 0; i < T; ++i)
+            for (int c = 0; c < D; ++c) {
+                av[c] += pc[i] * jb->dout[(size_t)i * D + c];
+                ak[c] += sc[i] * jb->q[(size_t)i * D + c];
+            }
+        for (int c = 0; c < D; ++c) {
+            jb->dv[(size_t)j * D + c] = av[c];
+            jb->dk[(size_t)j * D + c] = jb->scale * ak[c];
+        }
+    }
+    free(pc);
+    free(sc);
+    free(av);
+    free(ak);
+    return NULL;
+}
+
+/* Runs fn over nthreads jobs (job 0 on the calling thread). */
+static void run_head_pass(void *(*fn)(void *), head_bwd_job_t *jobs, int nthreads)
+{
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 1; t < nthreads; ++t)
+        pthread_create(&th[t], NULL, fn, &jobs[t]);
+    fn(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+}
+
+/* Gradients of one head on double inputs [T, D], the rows and then the keys
+ * split across nthreads threads. */
+static void head_bwd_threads(const double *q, const double *k, const double *v,
+                             const double *dout, int T, int D, int causal, double scale,
+                             double *dq, double *dk, double *dv, int nthreads)
+{
+    const size_t TT = (size_t)T * (size_t)T;
+    double *P = (double *)malloc(sizeof(double) * TT);
+    double *dS = (double *)malloc(sizeof(double) * TT);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > T) nthreads = T;
+    head_bwd_job_t *jobs = (head_bwd_job_t *)calloc((size_t)nthreads, sizeof(head_bwd_job_t));
+    for (int t = 0; t < nthreads; ++t) {
+        head_bwd_job_t j = {q, k, v, dout, T, D, causal, scale, P, dS, dq, dk, dv, t, nthreads};
+        jobs[t] = j;
+    }
+    run_head_pass(head_bwd_rows, jobs, nthreads);
+    run_head_pass(head_bwd_keys, jobs, nthreads);
+    free(jobs);
+    free(P);
+    free(dS);
+}
+
 /* Gradients of one head on double inputs: dq, dk, dv [T, D]. */
 void oracle_head_bwd_f64(const double *q, const double *k, const double *v, const double *dout,
                          int T, int D, int causal, double scale, double *dq, double *dk,
                          double *dv)
 {
-    const size_t TT = (size_t)T * (size_t)T;
-    double *P = (double *)malloc(sizeof(double) * TT);
-    double *dP = (double *)malloc(sizeof(double) * TT);
-    double *s = (double *)malloc(sizeof(double) * (size_t)T);
-    unsigned char *mk = (unsigned char *)malloc((size_t)T);
-    for (int i = 0; i < T; ++i) { /* S and P, row by row */
-        for (int j = 0; j < T; ++j) {
-            double acc = 0.0;
-            for (int c = 0; c < D; ++c)
-                acc += q[(size_t)i * D + c] * k[(size_t)j * D + c];
-            s[j] = scale * acc;
-            mk[j] = (unsigned char)(causal && j > i);
-        }
-        oracle_softmax_row(s, mk, T, P + (size_t)i * T);
-    }
-    for (int i = 0; i < T; ++i) /* dP = dO V^T */
-        for (int j = 0; j < T; ++j) {
-            double acc = 0.0;
-            for (int c = 0; c < D; ++c)
-                acc += dout[(size_t)i * D + c] * v[(size_t)j * D + c];
-            dP[(size_t)i * T + j] = acc;
-        }
-    for (int i = 0; i < T; ++i) { /* dS = P o (dP - rowsum(P o dP)), stored over dP */
-        double r = 0.0;
-        for (int j = 0; j < T; ++j)
-            r += P[(size_t)i * T + j] * dP[(size_t)i * T + j];
-        for (int j = 0; j < T; ++j)
-            dP[(size_t)i * T + j] = P[(size_t)i * T + j] * (dP[(size_t)i * T + j] - r);
-    }
-    for (int j = 0; j < T; ++j) /* dV = P^T dO, dK = scale dS^T Q */
-        for (int c = 0; c < D; ++c) {
-            double av = 0.0, ak = 0.0;
-            for (int i = 0; i < T; ++i) {
-                av += P[(size_t)i * T + j] * dout[(size_t)i * D + c];
-                ak += dP[(size_t)i * T + j] * q[(size_t)i * D + c];
-            }
-            dv[(size_t)j * D + c] = av;
-            dk[(size_t)j * D + c] = scale * ak;
-        }
-    for (int i = 0; i < T; ++i) /* dQ = scale dS K */
-        for (int c = 0; c < D; ++c) {
-            double acc = 0.0;
-            for (int j = 0; j < T; ++j)
-                acc += dP[(size_t)i * T + j] * k[(size_t)j * D + c];
-            dq[(size_t)i * D + c] = scale * acc;
-        }
-    free(P);
-    free(dP);
-    free(s);
-    free(mk);
+    head_bwd_threads(q, k, v, dout, T, D, causal, scale, dq, dk, dv, 1);
 }
 
 typedef struct {
@@ -327,6 +403,7 @@ typedef struct {
     double scale;
     double *dq, *dk, *dv;
     int tid, nthreads;
+    int inner;  /* threads inside one head (when there are fewer heads than threads) */
 } bwd_job_t;
 
 static void *bwd_worker(void *arg)
@@ -345,8 +422,8 @@ static void *bwd_worker(void *arg)
             k[e] = bf16_to_f64(jb->k[(size_t)kvh * n + e]);
             v[e] = bf16_to_f64(jb->v[(size_t)kvh * n + e]);
         }
-        oracle_head_bwd_f64(q, k, v, g, T, D, jb->causal, jb->scale, jb->dq + (size_t)bh * n, dk,
-                            dv);
+        head_bwd_threads(q, k, v, g, T, D, jb->causal, jb->scale, jb->dq + (size_t)bh * n, dk, dv,
+                         jb->inner);
         /* per query head: dk, dv of its K/V head; the caller sums over a group */
         memcpy(jb->dk + (size_t)bh * n, dk, sizeof(double) * n);
         memcpy(jb->dv + (size_t)bh * n, dv, sizeof(double) * n);
@@ -369,11 +446,16 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
         return -1;
     const int64_t BH = B * H;
     if (nthreads < 1) nthreads = 1;
-    if (nthreads > BH) nthreads = (int)BH;
+    int inner = 1;
+    if (nthreads > BH) { /* fewer heads than threads: heads one by one, split inside */
+        inner = nthreads;
+        nthreads = 1;
+    }
     bwd_job_t *jobs = (bwd_job_t *)calloc((size_t)nthreads, sizeof(bwd_job_t));
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     for (int t = 0; t < nthreads; ++t) {
-        bwd_job_t j = {q, k, v, dout, H, H / H_kv, BH, T, D, causal, scale, dq, dk, dv, t, nthreads};
+        bwd_job_t j = {q, k, v, dout, H, H / H_kv, BH, T, D, causal, scale, dq, dk, dv, t, nthreads,
+                       inner};
         jobs[t] = j;
     }
     for (int t = 1; t < nthreads; ++t)

@@ -137,8 +137,6 @@ def test_backward_rejects_bad_arguments(lib):
     ok = [A, A, A, A, A, A, A, A, A, A, 1, 4, 2, 256, 128, 1, 0.125, None]
     bad = list(ok); bad[9] = None            # no workspace
     assert lib.attn_bwd(*bad) == 1
-    bad = list(ok); bad[13] = 200            # T not a multiple of 128
-    assert lib.attn_bwd(*bad) == 3
     bad = list(ok); bad[12] = 3              # 4 heads over 3 K/V heads
     assert lib.attn_bwd(*bad) == 3
     bad = list(ok); bad[6] = A + 8           # misaligned dq
@@ -146,6 +144,8 @@ def test_backward_rejects_bad_arguments(lib):
     bad = list(ok); bad[14] = 80             # unsupported head size
     assert lib.attn_bwd(*bad) == 2
     assert attn.load_library().attn_bwd_workspace_bytes(2, 4, 256) == 2 * 4 * 256 * 8
+    # a ragged T is padded to whole 128-row blocks of statistics
+    assert attn.load_library().attn_bwd_workspace_bytes(2, 4, 200) == 2 * 4 * 256 * 8
 
 
 def test_decode_rejects_bad_arguments(lib):

@@ -52,13 +52,25 @@ def _run(B, H, H_kv, T, D, causal, seed, mult=1.0):
 
 
 CASES = [(1, 2, 2, 128, 64, True), (1, 2, 2, 256, 128, True), (2, 2, 2, 384, 64, False),
-         (1, 4, 2, 512, 128, True), (1, 2, 1, 256, 128, False), (1, 3, 3, 640, 128, True)]
+         (1, 4, 2, 512, 128, True), (1, 2, 1, 256, 128, False), (1, 3, 3, 640, 128, True),
+         # T not a multiple of 128: the last key/query block is padded inside attn_bwd
+         (1, 2, 2, 200, 64, True), (1, 2, 1, 333, 128, False),
+         (2, 2, 2, 1000, 128, True), (1, 3, 3, 129, 64, False), (1, 4, 2, 700, 64, True)]
 
 
 @pytest.mark.parametrize("B,H,H_kv,T,D,causal", CASES)
 def test_backward_every_element(B, H, H_kv, T, D, causal):
     errs = _run(B, H, H_kv, T, D, causal, 6000 + T + D + H)
     print(f"bwd B={B} H={H} H_kv={H_kv} T={T} D={D} causal={causal}: {errs}")
+    for name, (mx, mean) in errs.items():
+        assert mx <= MAX_REL and mean <= MEAN_REL, (name, mx, mean)
+
+
+def test_backward_bench_size_whole_head():
+    """One whole head at the size the backward is benchmarked on (T = 8192,
+    d_h = 128, causal): every element of dQ, dK and dV."""
+    errs = _run(1, 1, 1, 8192, 128, True, 6200)
+    print("bwd T=8192 d_h=128 causal, one head:", errs)
     for name, (mx, mean) in errs.items():
         assert mx <= MAX_REL and mean <= MEAN_REL, (name, mx, mean)
 

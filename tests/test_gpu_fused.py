@@ -59,6 +59,32 @@ def test_multi_head_logit_stress_every_element(D, seed):
         assert st["o_max_abs"] <= STRESS_O_MAX_ABS, st
 
 
+def _rising_scores(B, H, T, D, seed, slope):
+    """Q rows share one direction u; key j is slope * j * u plus unit noise, so
+    a row's scores climb with the key index by about slope * |u|^2 * scale per
+    key and the running maximum of every row jumps by far more than the lazy
+    rescale threshold (32 in log2 units) from one key tile to the next."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    u = torch.randn(D, generator=g)
+    q = (u + 0.1 * torch.randn(B, H, T, D, generator=g)).to(torch.bfloat16)
+    j = torch.arange(T, dtype=torch.float32).view(1, 1, T, 1)
+    k = (slope * j * u + torch.randn(B, H, T, D, generator=g)).to(torch.bfloat16)
+    v = torch.randn(B, H, T, D, generator=g).to(torch.bfloat16)
+    return q.contiguous(), k.contiguous(), v.contiguous()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+def test_rescale_path_every_element(D, causal):
+    """Every tile raises the row maximum past the threshold: the O rescale runs
+    on (nearly) every tile of every row."""
+    q, k, v = _rising_scores(1, 3, 1000, D, 9500 + D, slope=0.06)
+    st, _ = check_full(q, k, v, causal, 1 / math.sqrt(D))
+    print(f"rising D={D} causal={causal}", st)
+    assert_parity(st, f"rising D={D} causal={causal}")
+
+
 def test_tiny_workload_every_element():
     w = WORKLOADS["tiny_causal_T128_d64"]
     q, k, v = make_workload(w)
