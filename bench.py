@@ -471,10 +471,14 @@ def time_other(attn, w, dev, stream, args, local, peaks):
 
 def unfused_bytes(w) -> int:
     """Algorithmic HBM bytes of the materialised path per step: S written and
-    read, P written and read (bf16, T^2 per head each), plus Q, K, V read (K1
-    reads Q and K, K3 reads V), O written (bf16) and lse written (fp32)."""
+    read, P written and read (bf16; T^2 entries per head, or under the causal
+    mask the 128 x 128 tiles at or below the diagonal, which is all the path
+    moves), plus Q, K, V read (K1 reads Q and K, K3 reads V), O written (bf16)
+    and lse written (fp32)."""
     heads = w.B * w.H
-    return heads * (4 * w.T * w.T * 2 + 4 * w.T * w.D * 2 + w.T * 4)
+    nt = w.T // 128
+    entries = (nt * (nt + 1) // 2) * 128 * 128 if w.causal else w.T * w.T
+    return heads * (4 * entries * 2 + 4 * w.T * w.D * 2 + w.T * 4)
 
 
 def run_unfused(args, w, world, rank, local, peaks, peak_src):

@@ -12,6 +12,11 @@
 //   K2 softmax_kernel    P = softmax(mask(scale * S)), lse   (one warp per row,
 //                        warp-shuffle reduction of (max, sum) pairs)
 //   K3 pv_gemm_kernel    O = P V     (tcgen05, 128 x d_h tiles, 4-stage TMA ring)
+// Causal: what the mask hides is neither computed nor moved.  K1 skips the
+// 128 x 128 score tiles above the diagonal, K2 reads a row's scores only up
+// to the row itself and writes its probabilities up to the end of the row's
+// 128-row block (zeros past the diagonal), and K3 stops at each query
+// block's diagonal; the rest of S and P is left untouched.
 #pragma once
 
 #include "sm100.cuh"
@@ -49,6 +54,7 @@ __global__ void __launch_bounds__(128)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + 2 * TILE + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
+    if (p.causal && n0 > m0 + 127) return;  // every key of the tile is after every query
 
     if (threadIdx.x == 0) {
         mbar_init(b_load, 1);
@@ -141,9 +147,13 @@ __global__ void __launch_bounds__(256)
     const uint4 *src = reinterpret_cast<const uint4 *>(S + grow * (long long)T);
     uint4 *dst = reinterpret_cast<uint4 *>(P + grow * (long long)T);
     const int nchunk = T / 8;
+    // causal: scores are read up to the row itself, probabilities written up
+    // to the end of the row's 128-row block (what K3 multiplies)
+    const int rd_chunks = p.causal ? min(nchunk, (row >> 3) + 1) : nchunk;
+    const int wr_chunks = p.causal ? min(nchunk, ((row | 127) + 1) >> 3) : nchunk;
 
     float m = -INFINITY, l = 0.f;
-    for (int ch = lane; ch < nchunk; ch += 32) {
+    for (int ch = lane; ch < rd_chunks; ch += 32) {
         const uint4 v = src[ch];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         float x[8];
@@ -173,7 +183,11 @@ __global__ void __launch_bounds__(256)
         merge_ml(m, l, m2, l2);
     }
     const float inv_l = 1.f / l;
-    for (int ch = lane; ch < nchunk; ch += 32) {
+    for (int ch = lane; ch < wr_chunks; ch += 32) {
+        if (ch >= rd_chunks) {
+            dst[ch] = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
         const uint4 v = src[ch];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
@@ -227,7 +241,8 @@ __global__ void __launch_bounds__(128)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * 128, bh = blockIdx.y;
-    const int nchunks = p.T / 64;
+    // causal: the 64-key chunks up to this query block's diagonal
+    const int nchunks = p.causal ? min(p.T / 64, (m0 + 128) / 64) : p.T / 64;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NST; ++s) {

@@ -148,7 +148,11 @@ size_t attn_bwd_workspace_bytes(int B, int H, int T);
  *   K3 reads P and V and writes O = P V.
  *   s_ws, p_ws : caller-owned bf16 [B, H, T, T] workspaces (2 bytes per
  *                entry, the pages' convention), attn_unfused_workspace_bytes()
- *                bytes each; contents on return are S and P.
+ *                bytes each; contents on return are S and P -- under the
+ *                causal mask only what the mask leaves visible is computed and
+ *                moved: the 128 x 128 tiles of S at or below the diagonal, and
+ *                each row of P up to the end of its 128-row block (zeros past
+ *                the diagonal); the other entries are left as they were.
  * T must be a multiple of 128 on this path.  Other arguments as attn_fwd.
  */
 int attn_fwd_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
@@ -170,12 +174,12 @@ size_t attn_unfused_workspace_bytes(int B, int H, int T);
  *   Sizes: as attn_fwd_unfused, plus B * H * T * T <= 16,777,216 (for
  *   example one head at T = 4096, or 16 heads at T = 1024); larger problems
  *   return ATTN_ERR_WORKSPACE_LIMIT and launch nothing.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) for that device; make that first call before any
- *   stream capture.
+ *   The first call on a device (and the first after a change of its CUDA
+ *   context) looks up the array's device address (cudaGetSymbolAddress) for
+ *   that device; make that first call before any stream capture.
  *   Every call on a device shares the one array and leaves its S and P there;
- *   nothing in it needs to start at zero (each call writes all of S and P
- *   before reading them).  Calls whose work overlaps on the GPU (several
+ *   nothing in it needs to start at zero (each call writes every entry of S
+ *   and P that it later reads).  Calls whose work overlaps on the GPU (several
  *   streams, or several host threads) race on the array: serialise them.
  */
 int attn_fwd_unfused_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
