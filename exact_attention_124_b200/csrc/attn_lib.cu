@@ -316,9 +316,10 @@ template <int D>
 int launch_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
                    void *p_ws, int BH, int T, int causal, float scale, cudaStream_t stream)
 {
-    CUtensorMap mq, mk, mp, mv;
+    CUtensorMap mq, mk, ms, mp, mv;
     if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, BH, 128) ||
-        make_map(&mp, p_ws, T, T, BH, 128) || make_map(&mv, v, D, T, BH, 64))
+        make_map(&ms, s_ws, T, T, BH, 128) || make_map(&mp, p_ws, T, T, BH, 128) ||
+        make_map(&mv, v, D, T, BH, 64))
         return ATTN_ERR_LAUNCH;
     attn::UnfusedParams p;
     p.BH = BH;
@@ -328,7 +329,7 @@ int launch_unfused(const void *q, const void *k, const void *v, void *o, float *
     p.limit_ns = kWaitLimitNs;
     auto *S = static_cast<__nv_bfloat16 *>(s_ws);
     auto *P = static_cast<__nv_bfloat16 *>(p_ws);
-    attn::s_gemm_kernel<D><<<dim3(T / 128, T / 128, BH), 128, attn::K1_SMEM, stream>>>(mq, mk, S,
+    attn::s_gemm_kernel<D><<<dim3(T / 128, T / 128, BH), 128, attn::K1_SMEM, stream>>>(mq, mk, ms,
                                                                                       p);
     if (launch_status()) return ATTN_ERR_LAUNCH;
     const long long rows = (long long)BH * T;

@@ -37,12 +37,16 @@ constexpr int K1_SMEM = 1024 + 2 * 128 * 128 * 2 + 64;
 
 // ---------------------------------------------------------------------------
 // K1: one CTA per 128 x 128 tile of S (grid: T/128 key tiles, T/128 query
-// tiles, B*H heads); 128 threads.  S written raw (unscaled) as bf16.
+// tiles, B*H heads); 128 threads.  S written raw (unscaled) as bf16: each
+// thread packs its row into the shared memory the Q and K tiles used (two
+// 64-key boxes, 128-byte swizzled like a TMA load would write them, so the
+// 16-byte writes of a warp's 32 rows spread over all banks), then two TMA
+// stores move the tile out as whole 128-byte lines.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128)
     s_gemm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  __nv_bfloat16 *S, const UnfusedParams p)
+                  const __grid_constant__ CUtensorMap tmS, const UnfusedParams p)
 {
     constexpr int KB = D / 64, SUB = 128 * 128, TILE = 128 * D * 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -92,29 +96,39 @@ __global__ void __launch_bounds__(128)
     const bool w = mbar_wait(b_mma, 0, p.limit_ns, W_K1);
     ok = __all_sync(0xffffffffu, w) && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
-    if (ok) {
+    if (ok) {  // (the MMAs have completed: the Q and K tiles are no longer read)
         tc_fence_after_sync();
-        const int row = m0 + warp * 32 + lane;
+        const int r = warp * 32 + lane;  // row of the tile
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-        __nv_bfloat16 *dst_row = S + ((size_t)bh * p.T + row) * (size_t)p.T + n0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(taddr + 32 * c, r);
-            tmem_wait_ld_regs(r);
+        for (int c = 0; c < 4; ++c) {  // 32 keys; box c >> 1, 16-byte chunks 4 (c & 1) .. +3
+            uint32_t rg[32];
+            tmem_ld32(taddr + 32 * c, rg);
+            tmem_wait_ld_regs(rg);
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst_row + 32 * c);
+                pk[i] = pack_bf16x2(__uint_as_float(rg[2 * i]), __uint_as_float(rg[2 * i + 1]));
+            uint8_t *row_base = gbase + (c >> 1) * SUB + r * 128;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) {
+                const int chunk = 4 * (c & 1) + i;
+                *reinterpret_cast<uint4 *>(row_base + 16 * (chunk ^ (r & 7))) =
+                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
         }
+        fence_proxy_async_smem();
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    if (ok && threadIdx.x == 0) {
+        tma_store_3d(&tmS, base, n0, m0, bh);
+        tma_store_3d(&tmS, base + SUB, n0 + 64, m0, bh);
+        tma_store_commit();
+        tma_store_wait_read();  // the shared memory stays valid until the stores have read it
+    }
+    __syncwarp();  // warp 0 reconverges before the whole-warp dealloc
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
