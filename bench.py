@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other workloads (the per_config block)")
+    ap.add_argument("--no-other-paths", action="store_true",
+                    help="skip timing the backward, decode and unfused paths (the other_paths block)")
     ap.add_argument("--decode-tq", type=int, default=1, help="decode: new queries per head")
     ap.add_argument("--decode-hkv", type=int, default=0,
                     help="decode: K/V heads (0: the workload's H / 4)")
@@ -337,6 +339,21 @@ def run_ours(args):
             per_config[name] = time_other(attn, WORKLOADS[name], dev, stream, args, local, peaks)
             status |= attn.last_error()
 
+    # the other paths of the library on the same GPU, each timed like its own
+    # --path mode (backward and decode on this workload's shape; the unfused
+    # path on the two workloads whose S and P fit in a few GB)
+    other_paths = None
+    if world == 1 and not args.no_other_paths and args.workload == DEFAULT_WORKLOAD:
+        import argparse as _ap
+        sub = _ap.Namespace(**vars(args))
+        sub.steps, sub.warmup = max(3, min(args.steps, 10)), 3
+        other_paths = {"backward": run_backward(sub, w, 1, rank, local, peaks, peak_src, emit=False),
+                       "decode": run_decode(sub, w, 1, rank, local, peaks, peak_src, emit=False)}
+        for name in ("causal_T4096_d64", "full_T2048_d128_qk4"):
+            other_paths["unfused_" + name] = run_unfused(sub, WORKLOADS[name], 1, rank, local, peaks,
+                                                         peak_src, emit=False)
+        status |= attn.last_error()
+
     # end to end through the host-buffer C-ABI entry point
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     oh = torch.empty_like(qh).pin_memory()
@@ -391,6 +408,7 @@ def run_ours(args):
                          "launch_ms_min": min(per_launch)},
             "clocks": clocks,
             "per_config": per_config,
+            "other_paths": other_paths,
             "gpu_launches": launches,
             "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -481,7 +499,7 @@ def unfused_bytes(w) -> int:
     return heads * (4 * entries * 2 + 4 * w.T * w.D * 2 + w.T * 4)
 
 
-def run_unfused(args, w, world, rank, local, peaks, peak_src):
+def run_unfused(args, w, world, rank, local, peaks, peak_src, emit=True):
     import torch
     import exact_attention_124_b200 as attn
     dev = torch.device("cuda", local)
@@ -514,6 +532,13 @@ def run_unfused(args, w, world, rank, local, peaks, peak_src):
     nbytes = unfused_bytes(w)
     gbs = nbytes / (ms * 1e-3) / 1e9
     hbm = float(peaks["hbm_gbs"])
+    if not emit:
+        del S, P
+        torch.cuda.empty_cache()
+        return {"workload": w.name, "shape": w.describe(), "ms_per_step": ms,
+                "tflops": counted_flops(w) / (ms * 1e-3) / 1e12, "gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "algorithmic_bytes": nbytes, "launches": 3 * args.steps,
+                "clocks": sampler.summary(), "device_status": status}
     if rank == 0:
         line = {
             "metric": METRIC + " (unfused three-kernel path)", "path": "unfused",
@@ -533,7 +558,7 @@ def run_unfused(args, w, world, rank, local, peaks, peak_src):
     return 0 if status == 0 else 1
 
 
-def run_backward(args, w, world, rank, local, peaks, peak_src):
+def run_backward(args, w, world, rank, local, peaks, peak_src, emit=True):
     """Times attn_bwd (row statistics + dK/dV kernel + dQ kernel) per step.
     Counted FLOPs: 10*T^2*d_h per head (five T x T x d_h products: S, dP, dV,
     dK, dQ), halved when causal; the kernels actually run seven (S and dP are
@@ -570,6 +595,11 @@ def run_backward(args, w, world, rank, local, peaks, peak_src):
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     counted = 2.5 * counted_flops(w)
     peak = float(peaks["bf16_tflops"])
+    if not emit:
+        tf = counted / (ms * 1e-3) / 1e12
+        return {"workload": w.name, "shape": w.describe(), "ms_per_step": ms, "tflops_counted": tf,
+                "frac": tf / peak, "tflops_executed": 1.4 * tf, "launches": 3 * args.steps,
+                "clocks": sampler.summary(), "device_status": status}
     if rank == 0:
         value = whole_job_tflops(counted, world, ms)
         line = {
@@ -589,7 +619,7 @@ def run_backward(args, w, world, rank, local, peaks, peak_src):
     return 0 if status == 0 else 1
 
 
-def run_decode(args, w, world, rank, local, peaks, peak_src):
+def run_decode(args, w, world, rank, local, peaks, peak_src, emit=True):
     """Times attn_fwd_decode (split-KV partials + merge): --decode-tq queries
     per head against a K/V cache of the workload's T tokens with H_kv heads.
     HBM-bound: algorithmic bytes = the K/V cache read once + Q read + O, lse
@@ -640,6 +670,12 @@ def run_decode(args, w, world, rank, local, peaks, peak_src):
     nbytes = 2 * k.numel() * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     gbs = nbytes / (ms * 1e-3) / 1e9
     hbm = float(peaks["hbm_gbs"])
+    if not emit:
+        return {"workload": f"decode B={w.B} H={w.H} H_kv={H_kv} Tq={Tq} Tk={Tk} d_h={w.D} causal",
+                "us_per_step": 1e3 * ms, "gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "algorithmic_bytes": nbytes, "launches": 2 * args.steps,
+                "l2": "256 MB written, then 256 MB read, before each step",
+                "clocks": sampler.summary(), "device_status": status}
     if rank == 0:
         line = {
             "metric": "attention decode: effective HBM GB/s (K/V cache read once)",

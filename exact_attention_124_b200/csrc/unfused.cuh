@@ -23,6 +23,39 @@
 
 namespace attn {
 
+// TMA store helpers (only K1 stores through TMA).
+// 3-D tiled store of a box from shared memory at `src` to the tensor at
+// (x, y, z): x a multiple of 8 elements, every coordinate >= 0.  Tracked by
+// the issuing thread's bulk-async group (tma_store_commit / _wait_read).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y,
+                                             int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_commit()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until the committed stores have read their shared memory (it may then
+// be reused or released).
+__device__ __forceinline__ void tma_store_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Orders this thread's ordinary shared-memory writes before later accesses by
+// the asynchronous (TMA) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 struct UnfusedParams {
     int BH, T, causal;
     float c_log2;
