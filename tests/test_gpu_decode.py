@@ -62,6 +62,37 @@ def test_decode_every_element(B, H, H_kv, Tq, Tk, D, causal, splits):
     assert_parity(st, f"decode B={B} H={H} H_kv={H_kv} Tq={Tq} Tk={Tk} D={D} splits={splits}")
 
 
+def _rising_cache(B, H, H_kv, Tq, Tk, D, seed, slope=0.06):
+    """Queries share one direction u and cache key j is slope * j * u plus unit
+    noise: every row's running maximum jumps by far more than the lazy
+    rescale threshold (32 in log2 units) from one key tile to the next, in
+    every copy of the packed rows."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    u = torch.randn(D, generator=g)
+    q = (u + 0.1 * torch.randn(B, H, Tq, D, generator=g)).to(torch.bfloat16)
+    j = torch.arange(Tk, dtype=torch.float32).view(1, 1, Tk, 1)
+    k = (slope * j * u + torch.randn(B, H_kv, Tk, D, generator=g)).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, Tk, D, generator=g).to(torch.bfloat16)
+    return q.contiguous(), k.contiguous(), v.contiguous()
+
+
+@pytest.mark.parametrize("B,H,H_kv,Tq,Tk,D,splits", [
+    (1, 4, 1, 1, 1000, 128, 0),     # 4 packed rows: four copies of 32 keys per tile
+    (1, 4, 4, 40, 700, 64, -1),     # 40 rows: two copies of 64 keys, balanced partition
+    (1, 2, 1, 80, 900, 128, 2),     # 160 rows: two row blocks, one copy, fixed splits
+])
+def test_decode_rescale_path_every_element(B, H, H_kv, Tq, Tk, D, splits):
+    """The O rescale (which waits for the previous P.V) runs on nearly every tile."""
+    q, k, v = _rising_cache(B, H, H_kv, Tq, Tk, D, 7900 + Tq + D)
+    o, lse = attn.fwd_decode(*to_dev(q, k, v), True, splits=splits)
+    assert attn.last_error() == 0
+    ro, rl = oracle.attn_decode(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 1 / math.sqrt(D))
+    st = compare(o.double().cpu().numpy(), lse.double().cpu().numpy(), ro, rl)
+    print(f"decode rising Tq={Tq} D={D} splits={splits}", st)
+    assert_parity(st, f"decode rising Tq={Tq} D={D} splits={splits}")
+
+
 def test_decode_with_tq_equal_tk_matches_prefill():
     q, k, v = to_dev(*make_qkv(1, 4, 512, 128, 91))
     o1, l1 = attn.fwd(q, k, v, True)
