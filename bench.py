@@ -666,7 +666,10 @@ def run_decode(args, w, world, rank, local, peaks, peak_src, emit=True):
     torch.cuda.synchronize()
     sampler.stop()
     status = attn.last_error()
-    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world, dev)
+    # the mean, not the median: at tens of microseconds the event timestamps
+    # come in steps of about 2 us, and only the mean of many steps resolves
+    # differences below one step
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world, dev)
     nbytes = 2 * k.numel() * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     gbs = nbytes / (ms * 1e-3) / 1e9
     hbm = float(peaks["hbm_gbs"])

@@ -489,23 +489,39 @@ __global__ void __launch_bounds__(256)
         splits = dec_nseg(w, p.nkt, p.tot, p.G);
     }
     splits *= p.copies;  // every segment wrote one partial per copy of the rows
+    // Lane i holds partial s0 + i: the lse of up to 32 partials arrive in one
+    // round trip, the maximum by a shuffle butterfly, and the O loads below
+    // depend on nothing loaded before them.  A partial with lse = -inf (no
+    // visible key) gets weight 0; its O was written as exactly 0.
     float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[(size_t)s * nrows + r]);
+    for (int s0 = 0; s0 < splits; s0 += 32) {
+        const int s = s0 + lane;
+        if (s < splits) mx = fmaxf(mx, part_lse[(size_t)s * nrows + r]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     constexpr int PER = D / 32;
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
     float sum = 0.f;
     if (mx != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float ls = part_lse[(size_t)s * nrows + r];
-            if (ls == -INFINITY) continue;
-            const float w = expf(ls - mx);
-            sum += w;
-            const float *src = part_o + ((size_t)s * nrows + r) * D + lane * PER;
+        for (int s0 = 0; s0 < splits; s0 += 32) {
+            const int s = s0 + lane;
+            const float ls = s < splits ? part_lse[(size_t)s * nrows + r] : -INFINITY;
+            const float wl = ls == -INFINITY ? 0.f : expf(ls - mx);
+            sum += wl;
+            const int cnt = splits - s0 < 32 ? splits - s0 : 32;  // the same on every lane
+#pragma unroll 4
+            for (int i = 0; i < cnt; ++i) {
+                const float w = __shfl_sync(0xffffffffu, wl, i);
+                const float *src = part_o + ((size_t)(s0 + i) * nrows + r) * D + lane * PER;
 #pragma unroll
-            for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, src[i], acc[i]);
+                for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+            }
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     }
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
     __nv_bfloat16 *dst = o + r * D + lane * PER;
