@@ -487,8 +487,8 @@ int launch_decode(const void *q, const void *k, const void *v, void *o, float *l
     // its launch overlaps the partial kernel's tail and it waits on the device
     // (griddepcontrol.wait) until every partial result is written.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((nrows + 7) / 8));
-    cfg.blockDim = dim3(256);
+    cfg.gridDim = dim3((unsigned)((nrows + (128 / D) - 1) / (128 / D)));  // 128 / D rows per CTA
+    cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -467,19 +467,24 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 4) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-// One warp per query row: merge the segments' (O_s, lse_s) of its head.
+// The merge: 128 threads per CTA, 128 / D query rows per CTA, one thread per
+// output column.  Every thread walks the row's partials with loads that depend
+// on nothing loaded before them (the lse reads are the same address across
+// the row's threads: one broadcast each), so a row costs about two memory
+// round trips, and there are as many CTAs as rows x D / 128.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
     decode_combine_kernel(const DecodeParams p, __nv_bfloat16 *__restrict__ o, float *__restrict__ lse)
 {
     // launched as a programmatic dependent of decode_partial_kernel: wait
     // until that grid has finished and its writes are visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int ROWS = 128 / D;
     const long long nrows = p.nrows;
     const float *__restrict__ part_o = p.part_o;
     const float *__restrict__ part_lse = p.part_lse;
-    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    const long long r = (long long)blockIdx.x * ROWS + threadIdx.x / D;
+    const int c = threadIdx.x % D;
     if (r >= nrows) return;
     int splits = p.splits;
     if (p.balanced) {  // row (b, h, query) -> its head (K/V head, packed row block)
@@ -489,45 +494,23 @@ __global__ void __launch_bounds__(256)
         splits = dec_nseg(w, p.nkt, p.tot, p.G);
     }
     splits *= p.copies;  // every segment wrote one partial per copy of the rows
-    // Lane i holds partial s0 + i: the lse of up to 32 partials arrive in one
-    // round trip, the maximum by a shuffle butterfly, and the O loads below
-    // depend on nothing loaded before them.  A partial with lse = -inf (no
-    // visible key) gets weight 0; its O was written as exactly 0.
     float mx = -INFINITY;
-    for (int s0 = 0; s0 < splits; s0 += 32) {
-        const int s = s0 + lane;
-        if (s < splits) mx = fmaxf(mx, part_lse[(size_t)s * nrows + r]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    constexpr int PER = D / 32;
-    float acc[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    float sum = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[(size_t)s * nrows + r]);
+    float acc = 0.f, sum = 0.f;
     if (mx != -INFINITY) {
-        for (int s0 = 0; s0 < splits; s0 += 32) {
-            const int s = s0 + lane;
-            const float ls = s < splits ? part_lse[(size_t)s * nrows + r] : -INFINITY;
-            const float wl = ls == -INFINITY ? 0.f : expf(ls - mx);
-            sum += wl;
-            const int cnt = splits - s0 < 32 ? splits - s0 : 32;  // the same on every lane
-#pragma unroll 4
-            for (int i = 0; i < cnt; ++i) {
-                const float w = __shfl_sync(0xffffffffu, wl, i);
-                const float *src = part_o + ((size_t)(s0 + i) * nrows + r) * D + lane * PER;
-#pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, src[e], acc[e]);
-            }
+        // a partial with lse = -inf (no visible key) gets weight 0; its O was
+        // written as exactly 0
+#pragma unroll 8
+        for (int s = 0; s < splits; ++s) {
+            const float ls = part_lse[(size_t)s * nrows + r];
+            const float w = ls == -INFINITY ? 0.f : expf(ls - mx);
+            sum += w;
+            acc = fmaf(w, part_o[((size_t)s * nrows + r) * D + c], acc);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     }
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    __nv_bfloat16 *dst = o + r * D + lane * PER;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
-    if (lane == 0) lse[r] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    o[r * D + c] = __float2bfloat16_rn(sum > 0.f ? acc / sum : 0.f);
+    if (c == 0) lse[r] = sum > 0.f ? mx + logf(sum) : -INFINITY;
 }
 
 }  // namespace attn
