@@ -197,8 +197,8 @@ int device_ready(int *sms_out)
         ok &= set_smem(attn::decode_partial_kernel<128, 4>, attn::DecCfg<128>::SMEM);
         ok &= fused_all_ready<64>();
         ok &= fused_all_ready<128>();
-        ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1_SMEM);
-        ok &= set_smem(attn::s_gemm_kernel<128>, attn::K1_SMEM);
+        ok &= set_smem(attn::s_gemm_kernel<64>, attn::K1Cfg<64>::SMEM);
+        ok &= set_smem(attn::s_gemm_kernel<128>, attn::K1Cfg<128>::SMEM);
         ok &= set_smem(attn::pv_gemm_kernel<64>, attn::PvCfg<64>::SMEM);
         ok &= set_smem(attn::pv_gemm_kernel<128>, attn::PvCfg<128>::SMEM);
         ok &= set_smem(attn::selftest_qk_kernel<64>, 1024 + 2 * 128 * 64 * 2 + 64);
@@ -314,7 +314,7 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
 
 template <int D>
 int launch_unfused(const void *q, const void *k, const void *v, void *o, float *lse, void *s_ws,
-                   void *p_ws, int BH, int T, int causal, float scale, cudaStream_t stream)
+                   void *p_ws, int BH, int T, int causal, float scale, cudaStream_t stream, int sms)
 {
     CUtensorMap mq, mk, ms, mp, mv;
     if (make_map(&mq, q, D, T, BH, 128) || make_map(&mk, k, D, T, BH, 128) ||
@@ -329,8 +329,12 @@ int launch_unfused(const void *q, const void *k, const void *v, void *o, float *
     p.limit_ns = kWaitLimitNs;
     auto *S = static_cast<__nv_bfloat16 *>(s_ws);
     auto *P = static_cast<__nv_bfloat16 *>(p_ws);
-    attn::s_gemm_kernel<D><<<dim3(T / 128, T / 128, BH), 128, attn::K1_SMEM, stream>>>(mq, mk, ms,
-                                                                                      p);
+    {  // persistent: one CTA per SM over the tiles of S (under the causal mask, the lower ones)
+        const long long nt = T / 128;
+        const long long tiles = (causal ? nt * (nt + 1) / 2 : nt * nt) * BH;
+        const int grid = (int)(tiles < sms ? tiles : sms);
+        attn::s_gemm_kernel<D><<<grid, attn::K1Cfg<D>::THREADS, attn::K1Cfg<D>::SMEM, stream>>>(mq, mk, ms, p);
+    }
     if (launch_status()) return ATTN_ERR_LAUNCH;
     const long long rows = (long long)BH * T;
     attn::softmax_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(S, P, lse, p);
@@ -607,10 +611,11 @@ int attn_fwd_unfused(const void *q, const void *k, const void *v, void *o, float
     if (!s_ws || !p_ws) return ATTN_ERR_NULL;
     if (misaligned(s_ws) || misaligned(p_ws)) return ATTN_ERR_ALIGN;
     if (T % 128 != 0 || (long long)B * H > 65535) return ATTN_ERR_BAD_SHAPE;
-    if ((rc = device_ready(nullptr))) return rc;
+    int sms = 0;
+    if ((rc = device_ready(&sms))) return rc;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s)
-                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s);
+    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s, sms)
+                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s, sms);
 }
 
 int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
@@ -882,7 +887,8 @@ extern "C" int attn_fwd_unfused_noalloc(const void *q, const void *k, const void
     if (T % 128 != 0 || (long long)B * H > 65535) return ATTN_ERR_BAD_SHAPE;
     const unsigned long long one = (unsigned long long)B * H * T * (unsigned long long)T * 2ull;
     if (one > kNoallocBytes / 2) return ATTN_ERR_WORKSPACE_LIMIT;
-    if ((rc = device_ready(nullptr))) return rc;
+    int sms = 0;
+    if ((rc = device_ready(&sms))) return rc;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         (void)cudaGetLastError();
@@ -901,6 +907,6 @@ extern "C" int attn_fwd_unfused_noalloc(const void *q, const void *k, const void
     void *s_ws = ws;
     void *p_ws = ws + kNoallocBytes / 2;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s)
-                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s);
+    return d_h == 64 ? launch_unfused<64>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s, sms)
+                     : launch_unfused<128>(q, k, v, o, lse, s_ws, p_ws, B * H, T, causal, scale, s, sms);
 }

@@ -42,11 +42,17 @@ __device__ __forceinline__ void tma_store_commit()
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// Waits until the committed stores have read their shared memory (it may then
-// be reused or released).
-__device__ __forceinline__ void tma_store_wait_read()
+// Waits until at most the most recently committed store group has not yet
+// read its shared memory (every older group's source may be reused).
+__device__ __forceinline__ void tma_store_wait_read_1()
 {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Waits until every committed store has completed.
+__device__ __forceinline__ void tma_store_wait_all()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Orders this thread's ordinary shared-memory writes before later accesses by
@@ -64,105 +70,219 @@ struct UnfusedParams {
 
 enum : unsigned int { W_K1 = 32, W_K3_FULL, W_K3_EMPTY, W_K3_DONE };
 
-// K1 asks for the d_h = 128 footprint at both head sizes: at most three CTAs
-// per SM, so their 3 x 128 TMEM columns always fit in the SM's 512.
-constexpr int K1_SMEM = 1024 + 2 * 128 * 128 * 2 + 64;
-
 // ---------------------------------------------------------------------------
-// K1: one CTA per 128 x 128 tile of S (grid: T/128 key tiles, T/128 query
-// tiles, B*H heads); 128 threads.  S written raw (unscaled) as bf16: each
-// thread packs its row into the shared memory the Q and K tiles used (two
-// 64-key boxes, 128-byte swizzled like a TMA load would write them, so the
-// 16-byte writes of a warp's 32 rows spread over all banks), then two TMA
-// stores move the tile out as whole 128-byte lines.
+// K1: S = Q K^T, raw (unscaled) bf16, as a persistent kernel: one CTA per SM
+// walks the 128 x 128 tiles of S (all of them, or under the causal mask the
+// tiles at or below the diagonal), tile k*G + c for CTA c of G.  192 threads:
+//   warp 0     TMA producer: Q_m and K_n of each tile into a 2-stage ring
+//   warp 1     MMA issuer: S into one of two 128-column TMEM buffers
+//   warps 2-5  epilogue (thread = row = TMEM lane): TMEM -> bf16 -> one of two
+//              shared-memory staging tiles (128-byte swizzled, two 64-key
+//              boxes) -> two TMA stores, whole 128-byte lines
+// so loading tile k+1, computing it and storing tile k overlap.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(128)
+struct K1Cfg {
+    static constexpr int KB = D / 64;
+    static constexpr int SUB = 128 * 128;           // 128 rows x 128 bytes
+    static constexpr int TILE = 128 * D * 2;        // one Q or K tile
+    static constexpr int NST = 2;
+    static constexpr int STAGE = 2 * TILE;          // Q_m and K_n
+    static constexpr int STG = 128 * 128 * 2;       // one S tile (bf16)
+    static constexpr int OFF_STG = NST * STAGE;
+    static constexpr int OFF_BAR = OFF_STG + 2 * STG;
+    static constexpr int NBAR = 2 * NST + 5;        // full, empty, tfull[2], tempty[2], drain
+    static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 256;
+};
+
+// Tile l of a head's list -> (query block m, key block n).  Causal: the
+// lower triangle row by row, n <= m.
+__device__ __forceinline__ void k1_tile(const UnfusedParams &p, long long l, int nt, int &m, int &n)
+{
+    if (!p.causal) {
+        m = (int)(l / nt);
+        n = (int)(l - (long long)m * nt);
+        return;
+    }
+    int mm = (int)((sqrtf(8.f * (float)l + 1.f) - 1.f) * 0.5f);
+    while ((long long)(mm + 1) * (mm + 2) / 2 <= l) ++mm;
+    while ((long long)mm * (mm + 1) / 2 > l) --mm;
+    m = mm;
+    n = (int)(l - (long long)mm * (mm + 1) / 2);
+}
+
+// All 128 epilogue threads: true iff every one of them passes true.
+__device__ __forceinline__ bool epi_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
     s_gemm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmS, const UnfusedParams p)
 {
-    constexpr int KB = D / 64, SUB = 128 * 128, TILE = 128 * D * 2;
+    using C = K1Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base, sK = base + TILE;
-    const uint32_t b_load = base + 2 * TILE, b_mma = b_load + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + 2 * TILE + 16);
+    const uint32_t b_full = base + C::OFF_BAR;          // [NST]
+    const uint32_t b_empty = b_full + 8 * C::NST;       // [NST]
+    const uint32_t b_tfull = b_empty + 8 * C::NST;      // [2] S of TMEM buffer b computed
+    const uint32_t b_tempty = b_tfull + 16;             // [2] TMEM buffer b read out
+    const uint32_t b_drain = b_tempty + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
-    if (p.causal && n0 > m0 + 127) return;  // every key of the tile is after every query
+    const int G = (int)gridDim.x;
+    const int nt = p.T / 128;
+    const long long tph = p.causal ? (long long)nt * (nt + 1) / 2 : (long long)nt * nt;
+    const long long total = tph * p.BH;
+    const uint64_t lim = p.limit_ns;
 
     if (threadIdx.x == 0) {
-        mbar_init(b_load, 1);
-        mbar_init(b_mma, 1);
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(b_full + 8 * s, 1);
+            mbar_init(b_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_tfull + 8 * b, 1);
+            mbar_init(b_tempty + 8 * b, 128);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc(smem_addr(tmem_slot), 128);
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    bool ok = true;
-    if (threadIdx.x == 0) {
-        const uint64_t pol = policy_evict_last();
-        mbar_arrive_expect_tx(b_load, 2 * TILE);
-        for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(sQ + kb * SUB, &tmQ, b_load, 64 * kb, m0, bh, pol);
-            tma_load_3d(sK + kb * SUB, &tmK, b_load, 64 * kb, n0, bh, pol);
+    if (warp == 0) {
+        if (lane == 0) {  // TMA producer
+            const uint64_t pol = policy_evict_last();
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            int k = 0;
+            for (long long i = blockIdx.x; i < total; i += G, ++k) {
+                const int s = k % C::NST;
+                const uint32_t par = (uint32_t)(k / C::NST) & 1u;
+                if (!mbar_wait(b_empty + 8 * s, par ^ 1u, lim, W_K1, abort_flag)) { ok = false; break; }
+                const int bh = (int)(i / tph);
+                int m, n;
+                k1_tile(p, i - (long long)bh * tph, nt, m, n);
+                const uint32_t st = base + s * C::STAGE;
+                mbar_arrive_expect_tx(b_full + 8 * s, C::STAGE);
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (par << s);
+                for (int kb = 0; kb < C::KB; ++kb) {
+                    tma_load_3d(st + kb * C::SUB, &tmQ, b_full + 8 * s, 64 * kb, 128 * m, bh, pol);
+                    tma_load_3d(st + C::TILE + kb * C::SUB, &tmK, b_full + 8 * s, 64 * kb, 128 * n, bh, pol);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                for (int s = 0; s < C::NST; ++s)
+                    if ((armed >> s) & 1u) mbar_wait(b_full + 8 * s, (armed_par >> s) & 1u, lim, W_K1);
+            }
         }
-        ok = mbar_wait(b_load, 0, p.limit_ns, W_K1);
-        if (ok) {
-            tc_fence_after_sync();
+    } else if (warp == 1) {
+        if (lane == 0) {  // MMA issuer
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+            bool ok = true;
+            int k = 0;
+            for (long long i = blockIdx.x; i < total; i += G, ++k) {
+                const int s = k % C::NST, b = k & 1;
+                if (!(ok = mbar_wait(b_full + 8 * s, (uint32_t)(k / C::NST) & 1u, lim, W_K1, abort_flag)))
+                    break;
+                if (!(ok = mbar_wait(b_tempty + 8 * b, ((uint32_t)(k >> 1) & 1u) ^ 1u, lim, W_K1, abort_flag)))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t sq = base + s * C::STAGE, sk = sq + C::TILE;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * SUB + (kk & 3) * 32;
-                mma_ss(tmem, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024), idesc,
-                       kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::SUB + (kk & 3) * 32;
+                    mma_ss(tmem + 128 * b, sw128_desc(sq + off, 16, 1024), sw128_desc(sk + off, 16, 1024),
+                           idesc, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(b_empty + 8 * s);
+                tc_commit(b_tfull + 8 * b);
+            }
+            if (!ok) *abort_flag = 1;
+            tc_commit(b_drain);  // every MMA issued above has completed before TMEM is freed
+            mbar_wait(b_drain, 0, lim, W_K1);
+        }
+    } else {  // epilogue warpgroup: warps 2-5, TMEM lane quarter warp & 3
+        const int r = (warp & 3) * 32 + lane;  // row of the tile
+        const uint32_t taddr_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const bool storer = (warp == 2 && lane == 0);
+        int k = 0;
+        for (long long i = blockIdx.x; i < total; i += G, ++k) {
+            const int b = k & 1;
+            const bool w = mbar_wait(b_tfull + 8 * b, (uint32_t)(k >> 1) & 1u, lim, W_K1, abort_flag);
+            if (!epi_all(w)) {
+                if (threadIdx.x == 64) *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t rg[32];
+                tmem_ld32(taddr_lane + 128 * b + 32 * c, rg);
+                tmem_wait_ld_regs(rg);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[16 * c + e] = pack_bf16x2(__uint_as_float(rg[2 * e]), __uint_as_float(rg[2 * e + 1]));
+            }
+            tc_fence_before_sync();
+            mbar_arrive(b_tempty + 8 * b);  // TMEM buffer b may take the next tile
+            // staging buffer b: the store issued from it two tiles ago has read it
+            if (storer) tma_store_wait_read_1();
+            epi_sync();
+            uint8_t *stg = gbase + C::OFF_STG + b * C::STG;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {  // 16-byte chunk c: keys 8c .. 8c+7, box c / 8
+                uint8_t *row_base = stg + (c >> 3) * C::SUB + r * 128;
+                *reinterpret_cast<uint4 *>(row_base + 16 * ((c & 7) ^ (r & 7))) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            epi_sync();
+            if (storer) {
+                const int bh = (int)(i / tph);
+                int m, n;
+                k1_tile(p, i - (long long)bh * tph, nt, m, n);
+                const uint32_t sa = base + C::OFF_STG + b * C::STG;
+                tma_store_3d(&tmS, sa, 128 * n, 128 * m, bh);
+                tma_store_3d(&tmS, sa + C::SUB, 128 * n + 64, 128 * m, bh);
+                tma_store_commit();
             }
         }
-        tc_commit(b_mma);  // also covers the case with no MMA issued
-    }
-    __syncwarp();
-    const bool w = mbar_wait(b_mma, 0, p.limit_ns, W_K1);
-    ok = __all_sync(0xffffffffu, w) && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    ok = __syncthreads_and(ok ? 1 : 0) != 0;
-    if (ok) {  // (the MMAs have completed: the Q and K tiles are no longer read)
-        tc_fence_after_sync();
-        const int r = warp * 32 + lane;  // row of the tile
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 32 keys; box c >> 1, 16-byte chunks 4 (c & 1) .. +3
-            uint32_t rg[32];
-            tmem_ld32(taddr + 32 * c, rg);
-            tmem_wait_ld_regs(rg);
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(rg[2 * i]), __uint_as_float(rg[2 * i + 1]));
-            uint8_t *row_base = gbase + (c >> 1) * SUB + r * 128;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int chunk = 4 * (c & 1) + i;
-                *reinterpret_cast<uint4 *>(row_base + 16 * (chunk ^ (r & 7))) =
-                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-            }
-        }
-        fence_proxy_async_smem();
+        if (storer) tma_store_wait_all();  // the staging tiles stay valid until the stores finish
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (ok && threadIdx.x == 0) {
-        tma_store_3d(&tmS, base, n0, m0, bh);
-        tma_store_3d(&tmS, base + SUB, n0 + 64, m0, bh);
-        tma_store_commit();
-        tma_store_wait_read();  // the shared memory stays valid until the stores have read it
-    }
-    __syncwarp();  // warp 0 reconverges before the whole-warp dealloc
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------------------
