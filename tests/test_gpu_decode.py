@@ -3,7 +3,8 @@ oracle: Tq new queries against a Tk-token K/V cache, query i at position
 Tk - Tq + i ("FlashAttention -- avoid writing the giant intermediate": the
 persistent K/V state of cached decoding).  Same bounds as the prefill path.
 The cases cover fixed, balanced and automatic partitions and 1, 2 and 4
-copies of the packed query rows (more than 64, 33-64 and at most 32 rows)."""
+copies of the packed query rows (more than 64, 33-64 and at most 32 rows),
+including row counts that are not a multiple of the splits."""
 import math
 
 import numpy as np
@@ -56,6 +57,15 @@ def _case(B, H, H_kv, Tq, Tk, D, causal, splits, seed):
     (2, 8, 2, 12, 3000, 128, True, 0),
     (1, 16, 2, 5, 900, 64, False, -1),
     (1, 16, 2, 8, 260, 64, True, 3),
+    # 5 rows over 3 splits, 16 rows over 8, 1 row over 8
+    (1, 5, 1, 1, 3000, 128, True, 3),
+    (2, 16, 1, 1, 2000, 64, True, 8),
+    (1, 8, 8, 1, 1024, 128, False, 8),
+    # 24 rows (four copies): fixed splits and balanced
+    (2, 8, 2, 6, 1500, 128, True, 4),
+    (2, 8, 2, 6, 1500, 64, True, -1),
+    # 4 rows over 16 splits
+    (2, 8, 2, 1, 4096, 128, True, 16),
 ])
 def test_decode_every_element(B, H, H_kv, Tq, Tk, D, causal, splits):
     st = _case(B, H, H_kv, Tq, Tk, D, causal, splits, 7700 + Tq + Tk + D + splits)
@@ -79,6 +89,8 @@ def _rising_cache(B, H, H_kv, Tq, Tk, D, seed, slope=0.06):
 
 @pytest.mark.parametrize("B,H,H_kv,Tq,Tk,D,splits", [
     (1, 4, 1, 1, 1000, 128, 0),     # 4 packed rows: four copies of 32 keys per tile
+    (1, 4, 1, 1, 1000, 128, 2),     # the same over 2 fixed splits
+    (1, 8, 2, 6, 1100, 64, 3),      # 24 rows: four copies, 3 fixed splits
     (1, 4, 4, 40, 700, 64, -1),     # 40 rows: two copies of 64 keys, balanced partition
     (1, 2, 1, 80, 900, 128, 2),     # 160 rows: two row blocks, one copy, fixed splits
 ])
