@@ -319,29 +319,44 @@ __global__ void __launch_bounds__(256)
     const int rd_chunks = p.causal ? min(nchunk, (row >> 3) + 1) : nchunk;
     const int wr_chunks = p.causal ? min(nchunk, ((row | 127) + 1) >> 3) : nchunk;
 
+    // Each lane has U 16-byte loads in flight per step (the row's memory
+    // parallelism, not the exponentials, bounds this kernel).  Pass 1: the
+    // lane's online (max, sum) over its chunks; the second read of S is its
+    // last use (evict first).
+    constexpr int U = 4;
     float m = -INFINITY, l = 0.f;
-    for (int ch = lane; ch < rd_chunks; ch += 32) {
-        const uint4 v = src[ch];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float x[8];
+    for (int base = lane; base < rd_chunks; base += 32 * U) {
+        uint4 v[U];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[2 * i] = __uint_as_float(w[i] << 16) * c;
-            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * c;
+        for (int u = 0; u < U; ++u) {
+            const int ch = base + 32 * u;
+            v[u] = ch < rd_chunks ? src[ch] : make_uint4(0u, 0u, 0u, 0u);
         }
-        float cm = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (ch * 8 + i > lim_key) x[i] = -INFINITY;
-            cm = fmaxf(cm, x[i]);
+        for (int u = 0; u < U; ++u) {
+            const int ch = base + 32 * u;
+            if (ch >= rd_chunks) break;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[2 * i] = __uint_as_float(w[i] << 16) * c;
+                x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * c;
+            }
+            float cm = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (ch * 8 + i > lim_key) x[i] = -INFINITY;
+                cm = fmaxf(cm, x[i]);
+            }
+            if (cm == -INFINITY) continue;
+            const float mn = fmaxf(m, cm);
+            float add = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) add += fast_exp2(x[i] - mn);
+            l = l * fast_exp2(m - mn) + add;
+            m = mn;
         }
-        if (cm == -INFINITY) continue;
-        const float mn = fmaxf(m, cm);
-        float add = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) add += fast_exp2(x[i] - mn);
-        l = l * fast_exp2(m - mn) + add;
-        m = mn;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -350,26 +365,37 @@ __global__ void __launch_bounds__(256)
         merge_ml(m, l, m2, l2);
     }
     const float inv_l = 1.f / l;
-    for (int ch = lane; ch < wr_chunks; ch += 32) {
-        if (ch >= rd_chunks) {
-            dst[ch] = make_uint4(0u, 0u, 0u, 0u);
-            continue;
-        }
-        const uint4 v = src[ch];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+    // Pass 2: P, and zeros from the diagonal to the end of the row's block.
+    for (int base = lane; base < wr_chunks; base += 32 * U) {
+        uint4 v[U];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int k0 = ch * 8 + 2 * i;
-            const float a = (k0 > lim_key)
-                                ? 0.f
-                                : fast_exp2(__uint_as_float(w[i] << 16) * c - m) * inv_l;
-            const float b = (k0 + 1 > lim_key)
-                                ? 0.f
-                                : fast_exp2(__uint_as_float(w[i] & 0xFFFF0000u) * c - m) * inv_l;
-            o[i] = pack_bf16x2(a, b);
+        for (int u = 0; u < U; ++u) {
+            const int ch = base + 32 * u;
+            v[u] = ch < rd_chunks ? __ldcs(src + ch) : make_uint4(0u, 0u, 0u, 0u);
         }
-        dst[ch] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int ch = base + 32 * u;
+            if (ch >= wr_chunks) break;
+            if (ch >= rd_chunks) {
+                dst[ch] = make_uint4(0u, 0u, 0u, 0u);
+                continue;
+            }
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int k0 = ch * 8 + 2 * i;
+                const float a = (k0 > lim_key)
+                                    ? 0.f
+                                    : fast_exp2(__uint_as_float(w[i] << 16) * c - m) * inv_l;
+                const float b = (k0 + 1 > lim_key)
+                                    ? 0.f
+                                    : fast_exp2(__uint_as_float(w[i] & 0xFFFF0000u) * c - m) * inv_l;
+                o[i] = pack_bf16x2(a, b);
+            }
+            dst[ch] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
     if (lane == 0) lse[grow] = (m + fast_log2(l)) * 0.69314718055994530942f;
 }
