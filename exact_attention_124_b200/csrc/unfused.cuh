@@ -86,7 +86,7 @@ struct K1Cfg {
     static constexpr int KB = D / 64;
     static constexpr int SUB = 128 * 128;           // 128 rows x 128 bytes
     static constexpr int TILE = 128 * D * 2;        // one Q or K tile
-    static constexpr int NST = 2;
+    static constexpr int NST = D == 64 ? 4 : 2;  // Q/K stages: 4 x 32 KB at d_h = 64, 2 x 64 KB at 128
     static constexpr int STAGE = 2 * TILE;          // Q_m and K_n
     static constexpr int STG = 128 * 128 * 2;       // one S tile (bf16)
     static constexpr int OFF_STG = NST * STAGE;
