@@ -8,7 +8,8 @@
 // 2 * 2 * T^2 * 2 bytes per head through device memory that the fused kernel
 // never touches.  It exists to measure that traffic.
 //
-//   K1 s_gemm_kernel     S = Q K^T   (tcgen05, 128x128 tiles, TMA operands)
+//   K1 s_gemm_kernel     S = Q K^T   (tcgen05, 128x128 tiles, TMA operands;
+//                        persistent, one CTA per SM over the tiles)
 //   K2 softmax_kernel    P = softmax(mask(scale * S)), lse   (one warp per row,
 //                        warp-shuffle reduction of (max, sum) pairs)
 //   K3 pv_gemm_kernel    O = P V     (tcgen05, 128 x d_h tiles, 4-stage TMA ring)
@@ -74,7 +75,8 @@ enum : unsigned int { W_K1 = 32, W_K3_FULL, W_K3_EMPTY, W_K3_DONE };
 // K1: S = Q K^T, raw (unscaled) bf16, as a persistent kernel: one CTA per SM
 // walks the 128 x 128 tiles of S (all of them, or under the causal mask the
 // tiles at or below the diagonal), tile k*G + c for CTA c of G.  192 threads:
-//   warp 0     TMA producer: Q_m and K_n of each tile into a 2-stage ring
+//   warp 0     TMA producer: Q_m and K_n of each tile into a ring of NST
+//              stages (4 at d_h = 64, 2 at d_h = 128)
 //   warp 1     MMA issuer: S into one of two 128-column TMEM buffers
 //   warps 2-5  epilogue (thread = row = TMEM lane): TMEM -> bf16 -> one of two
 //              shared-memory staging tiles (128-byte swizzled, two 64-key
