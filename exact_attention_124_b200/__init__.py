@@ -8,7 +8,8 @@ library is missing every call raises.
 from ._lib import (AttnError, bwd, decode_plan, fused_plan, fwd, fwd_decode, fwd_gqa, fwd_host, fwd_unfused, last_error, library_path,
                    load_library, selftest_pv_tile, selftest_qk_tile, selftest_timeout,
                    set_exp_split, set_mma_order, status_str, fused_grid_ctas, unfused_workspace_bytes, version)
+from .autograd import attention
 
-__all__ = ["AttnError", "bwd", "decode_plan", "fused_plan", "fwd", "fwd_decode", "fwd_gqa", "fwd_host", "fwd_unfused", "last_error", "library_path",
+__all__ = ["AttnError", "attention", "bwd", "decode_plan", "fused_plan", "fwd", "fwd_decode", "fwd_gqa", "fwd_host", "fwd_unfused", "last_error", "library_path",
            "load_library", "selftest_pv_tile", "selftest_qk_tile", "selftest_timeout",
            "set_exp_split", "set_mma_order", "status_str", "fused_grid_ctas", "unfused_workspace_bytes", "version"]

@@ -153,7 +153,7 @@ def bwd(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, dq=None
         dv=None, ws=None, stream=None):
     """Backward pass: gradients (dq, dk, dv) from the forward's o and lse and
     the output gradient dout.  q/o/dout [B, H, T, d_h], k/v [B, H_kv, T, d_h],
-    T a multiple of 128."""
+    any T."""
     lib = load_library()
     B, H, T, D = _shape(q)
     H_kv = int(k.shape[1])
