@@ -1,8 +1,8 @@
 """Seeded random shapes through every GPU entry point, each checked against
 the float64 oracle with the bar of its own parity tests: grouped-query
-forward (any T, both d_h, causal or not), backward (T a
-multiple of 128, long enough for the K/V rings to wrap several times) and
-decode (fixed, balanced and automatic partitions, 1, 2 or 4 row copies)."""
+forward (any T, both d_h, causal or not), backward (long enough for the K/V
+rings to wrap several times, T a multiple of 128 or not) and decode (fixed,
+balanced and automatic partitions, 1, 2 or 4 row copies)."""
 import math
 import random
 
@@ -47,7 +47,10 @@ def test_random_forward(B, H, H_kv, T, D, causal, seed):
 
 
 BWD_CASES = [(1, 2, 1, 2048, 128, True, 32001), (1, 2, 2, 1536, 64, False, 32002),
-             (2, 4, 2, 1024, 128, True, 32003), (1, 3, 1, 1280, 64, True, 32004)]
+             (2, 4, 2, 1024, 128, True, 32003), (1, 3, 1, 1280, 64, True, 32004),
+             # ragged T: the last 128-row block of queries and keys is padded
+             (1, 2, 1, 1999, 128, True, 32005), (2, 2, 2, 777, 64, False, 32006),
+             (1, 4, 2, 1153, 128, False, 32007), (1, 2, 2, 321, 64, True, 32008)]
 
 
 @pytest.mark.parametrize("B,H,H_kv,T,D,causal,seed", BWD_CASES)
