@@ -142,15 +142,21 @@ bool set_smem(K kernel, int bytes)
 // The fused kernel re-balances registers with setmaxnreg; an increase that
 // the launch's registers cannot cover would wait forever, so refuse to launch
 // a build whose per-thread register count is below the split's assumption.
+template <int D, int EMU, bool CAUSAL>
+bool fused_ready1()
+{
+    using C = attn::FusedCfg<D>;
+    if (!set_smem(attn::attn_fwd_fused_kernel<D, EMU, CAUSAL>, CAUSAL ? C::SMEM : C::SMEM_NC)) return false;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn::attn_fwd_fused_kernel<D, EMU, CAUSAL>) != cudaSuccess)
+        return false;
+    return fa.numRegs >= C::REGS_LAUNCH && fa.maxThreadsPerBlock >= C::THREADS;
+}
+
 template <int D, int EMU>
 bool fused_ready()
 {
-    using C = attn::FusedCfg<D>;
-    if (!set_smem(attn::attn_fwd_fused_kernel<D, EMU>, C::SMEM)) return false;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn::attn_fwd_fused_kernel<D, EMU>) != cudaSuccess)
-        return false;
-    return fa.numRegs >= C::REGS_LAUNCH && fa.maxThreadsPerBlock >= C::THREADS;
+    return fused_ready1<D, EMU, true>() && fused_ready1<D, EMU, false>();
 }
 
 template <int D>
@@ -303,11 +309,20 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     p.lse = lse;
     const int grid = fused_grid(BH, T, causal, sms);
     const int split = g_exp_split >= 0 ? g_exp_split : (D == 64 ? kDefaultSplit64 : kDefaultSplit128);
-    switch (split) {
-        case 0: attn::attn_fwd_fused_kernel<D, 0><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
-        case 2: attn::attn_fwd_fused_kernel<D, 2><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
-        case 3: attn::attn_fwd_fused_kernel<D, 3><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
-        default: attn::attn_fwd_fused_kernel<D, 4><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+    if (causal) {
+        switch (split) {
+            case 0: attn::attn_fwd_fused_kernel<D, 0, true><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+            case 2: attn::attn_fwd_fused_kernel<D, 2, true><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+            case 3: attn::attn_fwd_fused_kernel<D, 3, true><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+            default: attn::attn_fwd_fused_kernel<D, 4, true><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
+        }
+    } else {
+        switch (split) {
+            case 0: attn::attn_fwd_fused_kernel<D, 0, false><<<grid, C::THREADS, C::SMEM_NC, stream>>>(mq, mk, mv, p); break;
+            case 2: attn::attn_fwd_fused_kernel<D, 2, false><<<grid, C::THREADS, C::SMEM_NC, stream>>>(mq, mk, mv, p); break;
+            case 3: attn::attn_fwd_fused_kernel<D, 3, false><<<grid, C::THREADS, C::SMEM_NC, stream>>>(mq, mk, mv, p); break;
+            default: attn::attn_fwd_fused_kernel<D, 4, false><<<grid, C::THREADS, C::SMEM_NC, stream>>>(mq, mk, mv, p); break;
+        }
     }
     return launch_status();
 }

@@ -118,6 +118,9 @@ struct FusedCfg {
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
     static constexpr int NBAR = 2 + 2 + 2 * NSTAGE + 2 + 4 + 2 + 1;
     static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    // non-causal instance: O staged through 4 KB per softmax warp, after the barriers
+    static constexpr int OFF_EPI = (OFF_BAR + NBAR * 8 + 16 + 1023) / 1024 * 1024;
+    static constexpr int SMEM_NC = 1024 + OFF_EPI + 8 * 4096;
     static constexpr int THREADS = 384;
     // setmaxnreg split: the launch gets 168 registers per thread (384 x 168 =
     // 64512); the control warpgroup gives back down to 88, the two softmax
@@ -246,7 +249,7 @@ struct Ring {
     }
 };
 
-template <int D, int EMU>
+template <int D, int EMU, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -534,9 +537,9 @@ __global__ void __launch_bounds__(384, 1)
                     for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r[i]);
                 }
                 const int key0 = 128 * j;
-                const bool need_mask = (p.causal && key0 + 127 > r0) || (key0 + 128 > p.T);
+                const bool need_mask = (CAUSAL && key0 + 127 > r0) || (key0 + 128 > p.T);
                 if (need_mask) {
-                    const int lim_key = p.causal ? min(row, p.T - 1) : p.T - 1;
+                    const int lim_key = CAUSAL ? min(row, p.T - 1) : p.T - 1;
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (key0 + c > lim_key) s[c] = -INFINITY;
@@ -624,6 +627,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after_sync();
             const float inv_l = 1.f / (l + lcor);
             const size_t orow = (size_t)u.bh * (size_t)p.T + (size_t)row;
+            if constexpr (CAUSAL) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
@@ -640,6 +644,43 @@ __global__ void __launch_bounds__(384, 1)
                     for (int i = 0; i < 4; ++i)
                         dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
+            }
+            } else {
+            // non-causal: O rows through this warp's 4 KB of shared memory, 64
+            // columns at a time, so that each store instruction writes four whole
+            // 128-byte lines (4 rows x 64 columns) instead of 32 scattered
+            // 16-byte pieces; 16-byte chunk j of a staged row sits at j ^ (row & 7)
+            uint8_t *stg = gbase + C::OFF_EPI + warp * 4096;
+            const int r0w = r0 + wq * 32;  // the warp's first row
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh) {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t rr[32];
+                    tmem_ld32(tO + 64 * hh + 32 * cc, rr);
+                    tmem_wait_ld_regs(rr);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * cc + jj;
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(rr[8 * jj + 0]) * inv_l, __uint_as_float(rr[8 * jj + 1]) * inv_l);
+                        v.y = pack_bf16x2(__uint_as_float(rr[8 * jj + 2]) * inv_l, __uint_as_float(rr[8 * jj + 3]) * inv_l);
+                        v.z = pack_bf16x2(__uint_as_float(rr[8 * jj + 4]) * inv_l, __uint_as_float(rr[8 * jj + 5]) * inv_l);
+                        v.w = pack_bf16x2(__uint_as_float(rr[8 * jj + 6]) * inv_l, __uint_as_float(rr[8 * jj + 7]) * inv_l);
+                        *reinterpret_cast<uint4 *>(stg + lane * 128 + 16 * (j ^ (lane & 7))) = v;
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const int rw = 4 * k4 + (lane >> 3), j = lane & 7;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stg + rw * 128 + 16 * (j ^ (rw & 7)));
+                    if (r0w + rw < p.T)
+                        *reinterpret_cast<uint4 *>(p.o + ((size_t)u.bh * (size_t)p.T + (size_t)(r0w + rw)) * D +
+                                                   64 * hh + 8 * j) = v;
+                }
+                __syncwarp();
+            }
             }
             if (row < p.T) p.lse[orow] = (m + fast_log2(l)) * 0.69314718055994530942f;
             tc_fence_before_sync();
