@@ -64,20 +64,26 @@ bool driver_fn(const char *name, F &out)
 }
 
 // Process-unique id of the current device's context (creating the primary
-// context if none is current yet); 0 on failure.
+// context if none is current yet); 0 on failure.  Makes no runtime call while
+// a context is current, so the entry points can be captured into a CUDA graph
+// (stream capture forbids cudaFree, the usual way to bind the context).
 unsigned long long current_ctx_id()
 {
-    if (cudaFree(nullptr) != cudaSuccess) {  // makes the runtime bind its primary context
-        (void)cudaGetLastError();
-        return 0;
-    }
     if (!driver_fn("cuCtxGetCurrent", g_ctx_get_current) || !driver_fn("cuCtxGetId", g_ctx_get_id))
         return 0;
     CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return 0;
+    if (ctx == nullptr) {
+        // no context on this thread yet (never the case during a capture):
+        // make the runtime bind its primary context
+        if (cudaFree(nullptr) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return 0;
+        }
+        if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    }
     unsigned long long id = 0;
-    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
-        g_ctx_get_id(ctx, &id) != CUDA_SUCCESS)
-        return 0;
+    if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
     return id;
 }
 
