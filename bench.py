@@ -702,27 +702,40 @@ def run_decode(args, w, world, rank, local, peaks, peak_src, emit=True):
     # step, same events) replayed from a CUDA graph that holds its two launches,
     # as a decode loop would run it; the host-side launch path is then off the
     # timed critical path.
+    # (A failed capture is reported in this entry and does not end the run.)
     g = torch.cuda.CUDAGraph()
     torch.cuda.synchronize()
-    with torch.cuda.graph(g):
-        attn.fwd_decode(q, k, v, True, w.scale, splits=0, o=o, lse=lse, ws=ws)
-    for _ in range(3):
-        g.replay()
-    gevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
+    try:
+        with torch.cuda.graph(g):
+            attn.fwd_decode(q, k, v, True, w.scale, splits=0, o=o, lse=lse, ws=ws)
+        captured = None
+    except Exception as e:  # noqa: BLE001 -- reported, not hidden
+        captured = f"{type(e).__name__}: {e}".splitlines()[0][:200]
     torch.cuda.synchronize()
-    for a, b in gevs:
-        flush.zero_()
-        torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
-        a.record(stream)
-        g.replay()
-        b.record(stream)
-    torch.cuda.synchronize()
-    status = status or attn.last_error()
-    gms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in gevs), world, dev)
+    if captured is None:
+        for _ in range(3):
+            g.replay()
+        gevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in gevs:
+            flush.zero_()
+            torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        status = status or attn.last_error()
+        gms = statistics.mean(a.elapsed_time(b) for a, b in gevs)
+    else:
+        gms = float("nan")
+    # every rank takes the same collective step, captured or not
+    gms = max_over_ranks(gms, world, dev)
     gg = nbytes / (gms * 1e-3) / 1e9
     graphed = {"us_per_step": 1e3 * gms, "gbs": gg, "frac_of_hbm": gg / hbm, "steps": args.steps,
                "l2": "256 MB written, then 256 MB read, before each step"}
+    if captured is not None:
+        graphed = {"error": captured}
     del g
     if not emit:
         return {"workload": f"decode B={w.B} H={w.H} H_kv={H_kv} Tq={Tq} Tk={Tk} d_h={w.D} causal",
