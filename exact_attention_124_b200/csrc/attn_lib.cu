@@ -315,6 +315,11 @@ int launch_fused(const void *q, const void *k, const void *v, void *o, float *ls
     p.lse = lse;
     const int grid = fused_grid(BH, T, causal, sms);
     const int split = g_exp_split >= 0 ? g_exp_split : (D == 64 ? kDefaultSplit64 : kDefaultSplit128);
+    // One kernel instance per mask mode.  The causal one stores each thread's O
+    // row straight to global memory; the non-causal one passes a warp's rows
+    // through shared memory (whole 128-byte lines per store) and needs the
+    // larger shared-memory size.  The causal kernel is faster with the direct
+    // stores: its epilogue timing keeps the two warpgroups out of step.
     if (causal) {
         switch (split) {
             case 0: attn::attn_fwd_fused_kernel<D, 0, true><<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p); break;
