@@ -35,10 +35,12 @@
  *    are read with attn_last_error().
  *  - Results are deterministic run to run.  The library is thread-compatible,
  *    not thread-safe: serialise concurrent calls from several host threads.
- *  - attn_fwd, attn_fwd_gqa, attn_fwd_decode and attn_bwd may be captured
- *    into a CUDA graph (stream capture) once a first call has done the
- *    device set-up in that context: they then only launch kernels on
- *    `stream`.  attn_last_error synchronises and must not be captured.
+ *  - attn_fwd, attn_fwd_gqa, attn_fwd_decode, attn_bwd, attn_fwd_unfused and
+ *    attn_fwd_host may be captured into a CUDA graph (stream capture) once a
+ *    first call has done the device set-up in that context: they then only
+ *    launch kernels and copies on `stream` (attn_fwd_host: on its own two
+ *    streams, forked from and joined back to `stream` through events).
+ *    attn_last_error synchronises and must not be captured.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H

@@ -100,3 +100,44 @@ def test_backward_graph_replay_matches_direct_call():
         _replay(g)
         ref = attn.bwd(q, k, v, o, lse, do, True)
         assert all(torch.equal(a, b) for a, b in zip((dq, dk, dv), ref))
+
+
+def test_unfused_graph_replay_matches_direct_call():
+    # three kernels (S to memory, softmax, P.V) in one graph
+    B, H, T, D = 1, 2, 256, 64
+    q, k, v = (_randn((B, H, T, D), 100 + i) for i in range(3))
+    o_ref, lse_ref, _, _ = attn.fwd_unfused(q, k, v, True)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    s_ws = torch.empty((B, H, T, T), dtype=torch.bfloat16, device=q.device)
+    p_ws = torch.empty_like(s_ws)
+    g = _capture(lambda: attn.fwd_unfused(q, k, v, True, o=o, lse=lse, s_ws=s_ws, p_ws=p_ws))
+    for step in range(2):
+        if step:
+            k.copy_(_randn((B, H, T, D), 103, 2.0))
+            o_ref, lse_ref, _, _ = attn.fwd_unfused(q, k, v, True)
+        _replay(g)
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+def test_host_buffer_forward_graph_replay():
+    # the copies run on the library's own two streams, forked from and joined
+    # back to the capturing stream through events, so the graph holds them too
+    B, H, T, D = 1, 3, 200, 128
+    q, k, v = (_randn((B, H, T, D), 110 + i) for i in range(3))
+    qh, kh, vh = [t.cpu().pin_memory() for t in (q, k, v)]
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((B, H, T), dtype=torch.float32).pin_memory()
+    dq, dk, dv, do_ = (torch.empty_like(q) for _ in range(4))
+    dl = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    attn.fwd_host(qh, kh, vh, oh, lh, dq, dk, dv, do_, dl, True)  # set-up: streams, events
+    torch.cuda.synchronize()
+    g = _capture(lambda: attn.fwd_host(qh, kh, vh, oh, lh, dq, dk, dv, do_, dl, True))
+    for step in range(2):
+        if step:
+            qh.copy_(_randn((B, H, T, D), 113, 2.0).cpu())
+        oh.zero_()
+        lh.zero_()
+        _replay(g)
+        o_ref, lse_ref = attn.fwd(qh.cuda(), kh.cuda(), vh.cuda(), True)
+        assert torch.equal(oh, o_ref.cpu()) and torch.equal(lh, lse_ref.cpu())
